@@ -1,0 +1,263 @@
+"""CPU oracle for the QuaRot online rotation + INT4 hot path (numpy front end).
+
+TEST INFRASTRUCTURE ONLY: the test suite, the smoke check and the CPU-baseline
+leg of the benchmark may import this package; the product library never does.
+It is independent of the CUDA library (no shared code, headers or tables).
+The arithmetic lives in quarot_oracle.c (fp64 / int64); this module only
+marshals numpy arrays into it and composes its steps in the method's order:
+
+    x' = (x * diag(s)) * H / sqrt(n)             randomized Hadamard rotation
+    s_x = max|x'| / 7, q = clamp(rint(x'/s), -8, 7)   symmetric INT4 RTN
+    pack: byte i = q[2i] (bits 0-3) | q[2i+1] (bits 4-7)
+    acc = qa . qw^T  (int64), y = acc * s_x[t] * s_w[n]  (fp64, then fp16)
+
+Sources: QuaRot (ISTA record abstract; Elamur Research summary, "Summary" and
+"Key points"), the onlyaistuff.com QuaRot article (randomized Hadamard), and
+DuQuant (chapterpal) Knowl 1, 2 and 12 for invariance, block-128 rotations and
+the per-head Hadamard on the attention path.  Each C function states the
+reading it takes where the pages are silent.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build_oracle
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = build_oracle.build()
+        L = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        sigs = {
+            "qo_sylvester": [I64, P],
+            "qo_fwht": [P, I64],
+            "qo_rotate": [P, I64, I64, P, I64, P],
+            "qo_rotate_dense": [P, I64, I64, P, I64, P],
+            "qo_quantize": [P, I64, I64, I64, P, P, P],
+            "qo_pack": [P, I64, P],
+            "qo_unpack": [P, I64, P],
+            "qo_int_gemm": [P, P, I64, I64, I64, I64, P],
+            "qo_dequant_linear": [P, I64, I64, I64, P, P, P, P],
+            "qo_kv_quant": [P, P, I64, I64, I64, I64, P, P, P, P, P],
+            "qo_kv_scores": [P, I64, I64, I64, I64, I64, P, P, P, P],
+            "qo_f16_to_f64_array": [P, I64, P],
+            "qo_f64_to_f16_array": [P, I64, P],
+            "qo_max_threads": [],
+        }
+        for name, args in sigs.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = ctypes.c_int
+        L.qo_f16_to_f64_array.restype = None
+        L.qo_f64_to_f16_array.restype = None
+        _lib = L
+    return _lib
+
+
+def _p(a):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise ValueError(f"oracle {what} rejected its arguments (rc={rc})")
+
+
+def max_threads() -> int:
+    return int(lib().qo_max_threads())
+
+
+# --- fp16 ------------------------------------------------------------------
+
+def f16_bits(x):
+    """fp16 array (or bits) -> uint16 bit patterns."""
+    x = np.asarray(x)
+    if x.dtype == np.float16:
+        return np.ascontiguousarray(x).view(np.uint16)
+    return _c(x, np.uint16)
+
+
+def f16_to_f64(bits):
+    b = f16_bits(bits)
+    out = np.empty(b.shape, np.float64)
+    lib().qo_f16_to_f64_array(_p(b), b.size, _p(out))
+    return out
+
+
+def f64_to_f16(x):
+    x = _c(x, np.float64)
+    out = np.empty(x.shape, np.uint16)
+    lib().qo_f64_to_f16_array(_p(x), x.size, _p(out))
+    return out
+
+
+# --- rotation --------------------------------------------------------------
+
+def sylvester(n: int) -> np.ndarray:
+    H = np.empty((n, n), np.int8)
+    _check(lib().qo_sylvester(n, _p(H)), "sylvester")
+    return H
+
+
+def fwht(v) -> np.ndarray:
+    """Unnormalized transform of each row of v (last axis, power-of-two length)."""
+    v = _c(v, np.float64).copy()
+    n = v.shape[-1]
+    flat = v.reshape(-1, n)
+    for r in range(flat.shape[0]):
+        row = flat[r]
+        _check(lib().qo_fwht(_p(row), n), "fwht")
+    return v
+
+
+def rotate(x16, signs, had_block: int = 0, dense: bool = False) -> np.ndarray:
+    """x' = (x * diag(s)) * R for each row of the fp16 matrix x16 [M, K]."""
+    xb = f16_bits(x16)
+    M, K = xb.shape
+    s = _c(signs, np.int8)
+    assert s.shape == (K,)
+    out = np.empty((M, K), np.float64)
+    fn = lib().qo_rotate_dense if dense else lib().qo_rotate
+    _check(fn(_p(xb), M, K, _p(s), had_block, _p(out)), "rotate")
+    return out
+
+
+# --- quantizer -------------------------------------------------------------
+
+def quantize(xr, group: int = 0):
+    """Returns (codes int8 [M, K], scales): fp64 [M] if group == 0, else fp16 bits [M, K/group]."""
+    xr = _c(xr, np.float64)
+    M, K = xr.shape
+    codes = np.empty((M, K), np.int8)
+    if group == 0:
+        sc = np.empty((M,), np.float64)
+        _check(lib().qo_quantize(_p(xr), M, K, 0, _p(codes), _p(sc), None), "quantize")
+    else:
+        sc = np.empty((M, K // group), np.uint16)
+        _check(lib().qo_quantize(_p(xr), M, K, group, _p(codes), None, _p(sc)), "quantize")
+    return codes, sc
+
+
+def pack(codes) -> np.ndarray:
+    c = _c(codes, np.int8)
+    out = np.empty(c.shape[:-1] + (c.shape[-1] // 2,), np.uint8)
+    _check(lib().qo_pack(_p(c), c.size, _p(out)), "pack")
+    return out
+
+
+def unpack(packed) -> np.ndarray:
+    p = _c(packed, np.uint8)
+    out = np.empty(p.shape[:-1] + (p.shape[-1] * 2,), np.int8)
+    _check(lib().qo_unpack(_p(p), p.size * 2, _p(out)), "unpack")
+    return out
+
+
+def rotate_quant(x16, signs, had_block: int = 0, group: int = 0):
+    """The full activation step: rotate, quantize, pack.  Returns (packed, scales, x')."""
+    xr = rotate(x16, signs, had_block)
+    codes, sc = quantize(xr, group)
+    return pack(codes), sc, xr
+
+
+# --- integer product -------------------------------------------------------
+
+def int_gemm(qa, qw, group: int = 0) -> np.ndarray:
+    """acc[m, n(, g)] = sum_k qa[m, k] qw[n, k] over each group (int64)."""
+    qa = _c(qa, np.int8)
+    qw = _c(qw, np.int8)
+    M, K = qa.shape
+    N, K2 = qw.shape
+    assert K == K2
+    G = 1 if group == 0 else K // group
+    acc = np.empty((M, N, G), np.int64)
+    _check(lib().qo_int_gemm(_p(qa), _p(qw), M, N, K, group, _p(acc)), "int_gemm")
+    return acc[:, :, 0] if group == 0 else acc
+
+
+def scales_to_f64(sc):
+    """fp64 scales pass through; fp16 bit patterns (or fp16 arrays) decode exactly."""
+    sc = np.asarray(sc)
+    if sc.dtype in (np.uint16, np.float16):
+        return f16_to_f64(sc)
+    return _c(sc, np.float64)
+
+
+def dequant_linear(acc, sa, sw, group: int = 0):
+    """y = acc * sa[m] * sw[n] (or the group sum).  Returns (y fp64, y fp16 bits)."""
+    acc = np.asarray(acc, np.int64)
+    if group == 0:
+        M, N = acc.shape
+        G = 1
+        acc = acc.reshape(M, N, 1)
+    else:
+        M, N, G = acc.shape
+    acc = _c(acc, np.int64)
+    sa64 = scales_to_f64(sa).reshape(M, G)
+    sw64 = scales_to_f64(sw).reshape(N, G)
+    sa64 = _c(sa64, np.float64)
+    sw64 = _c(sw64, np.float64)
+    y = np.empty((M, N), np.float64)
+    y16 = np.empty((M, N), np.uint16)
+    _check(lib().qo_dequant_linear(_p(acc), M, N, G, _p(sa64), _p(sw64), _p(y), _p(y16)),
+           "dequant_linear")
+    return y, y16
+
+
+def weight_prep(w16, signs, had_block: int = 0, group: int = 0):
+    """Offline weight step: rotate the rows of W with the same signs and Hadamard
+    (QuaRot summary: most rotations are fused into the weights), then quantize
+    per output channel (group 0) or per 128-group.  Returns (packed, scales)."""
+    packed, sc, _ = rotate_quant(w16, signs, had_block, group)
+    return packed, sc
+
+
+def linear(x16, w16, signs, had_block: int = 0, group: int = 0):
+    """The whole prefill linear: both operands rotated and quantized, then the
+    integer product and the dequantized fp16 output."""
+    qa_p, sa, _ = rotate_quant(x16, signs, had_block, group)
+    qw_p, sw = weight_prep(w16, signs, had_block, group)
+    acc = int_gemm(unpack(qa_p), unpack(qw_p), group)
+    y, y16 = dequant_linear(acc, sa, sw, group)
+    return dict(qa=qa_p, sa=sa, qw=qw_p, sw=sw, acc=acc, y=y, y16=y16)
+
+
+# --- KV cache --------------------------------------------------------------
+
+def kv_quant(k16, v16, signs):
+    """k16, v16: fp16 [B, T, H, D]; signs [H, D].  Returns packed codes and fp16-bit scales."""
+    kb = f16_bits(k16)
+    vb = f16_bits(v16)
+    B, T, H, D = kb.shape
+    s = _c(signs, np.int8)
+    assert s.shape == (H, D)
+    kc = np.empty((B, T, H, D), np.int8)
+    vc = np.empty((B, T, H, D), np.int8)
+    ks = np.empty((B, T, H), np.uint16)
+    vs = np.empty((B, T, H), np.uint16)
+    _check(lib().qo_kv_quant(_p(kb), _p(vb), B, T, H, D, _p(s), _p(kc), _p(ks), _p(vc), _p(vs)),
+           "kv_quant")
+    return pack(kc), ks, pack(vc), vs
+
+
+def kv_scores(q16, signs, kq_packed, ks):
+    """q16 fp16 [B, Hq, D]; kq_packed [B, T, H, D/2]; ks fp16 bits [B, T, H] -> fp64 [B, Hq, T]."""
+    qb = f16_bits(q16)
+    B, Hq, D = qb.shape
+    kc = unpack(kq_packed)
+    _, T, H, _ = kc.shape
+    s = _c(signs, np.int8)
+    ks64 = _c(scales_to_f64(ks), np.float64)
+    out = np.empty((B, Hq, T), np.float64)
+    _check(lib().qo_kv_scores(_p(qb), B, Hq, H, D, T, _p(s), _p(kc), _p(ks64), _p(out)),
+           "kv_scores")
+    return out

@@ -1,0 +1,436 @@
+/*
+ * quarot_oracle.c -- plain CPU oracle for the QuaRot online rotation + INT4 path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path links, loads or calls
+ * this file.  Only the test suite, the smoke check and the CPU-baseline leg of
+ * the benchmark use it.  It shares no code, header, table or helper with the
+ * CUDA library: it is a second, independent statement of what the path
+ * computes, written for reading, not for speed.
+ *
+ * Arithmetic: fp64 for every real number, int64 for every integer sum.
+ * Parallelism: OpenMP over independent rows only; no blocking, no fusion and
+ * no reordering of any sum beyond what each definition below states.
+ *
+ * What it follows:
+ *  - QuaRot: Outlier-free 4-bit inference in rotated LLMs (ISTA research
+ *    explorer record, abstract): weights, activations and the KV cache are
+ *    quantized to 4 bits and all matrix products run in 4 bits; the rotation
+ *    leaves the layer output unchanged (computational invariance).
+ *  - QuaRot: Outlier-Free 4-Bit Inference in Rotated LLMs (Elamur Research
+ *    summary), "Summary": the model is multiplied by random orthogonal
+ *    Hadamard matrices, most folded into the weights, a few applied online;
+ *    "Key points": activations are quantized on the fly with round-to-nearest,
+ *    and a group-wise variant uses groups of 128.
+ *  - Scientists from ETH Zurich, EPFL and Microsoft have presented QuaRot
+ *    (onlyaistuff.com article): the rotations are randomized Hadamard
+ *    transformations.
+ *  - DuQuant: Distributing Outliers via Dual Transformation Makes Stronger
+ *    Quantized LLMs (chapterpal), Knowl 1 (Y = XW = (XG)(G^-1 W)), Knowl 2
+ *    (block-diagonal rotations of size 2^n; a normalized Hadamard has a
+ *    uniform first row), Knowl 12 (block size 128; a fixed Hadamard with
+ *    entries +-1/sqrt(2^n) on the attention path, per-head quantization).
+ *
+ * Readings where the pages are silent (each is also listed in the design
+ * notes): Sylvester order for H_n, normalization 1/sqrt(n), signs applied
+ * before the Hadamard (x * diag(s) * H), symmetric scale absmax/7, codes
+ * clamp(rint(v/scale), -8, 7) with round-half-to-even, a zero stored scale
+ * giving zero codes, group scales stored as fp16 and the stored fp16 value
+ * used to quantize, nibble order low = even element.
+ *
+ * Parity pins: every function here is pinned by a CPU test against something
+ * other than itself (textbook Sylvester matrices, scipy's Hadamard, closed
+ * forms, numpy's fp16 conversion, brute-force integer loops, invariants).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------------ */
+/* IEEE binary16 <-> binary64, written from the format's definition.          */
+/* ------------------------------------------------------------------------ */
+
+/* Exact value of a binary16 bit pattern. */
+double qo_f16_to_f64(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int exp = (h >> 10) & 0x1f;
+    int man = h & 0x3ff;
+    double v;
+    if (exp == 0) {
+        v = ldexp((double)man, -24);                 /* subnormal: man * 2^-24 */
+    } else if (exp == 31) {
+        v = man ? NAN : INFINITY;
+    } else {
+        v = ldexp((double)(1024 + man), exp - 25);   /* (1 + man/1024) * 2^(exp-15) */
+    }
+    return sign ? -v : v;
+}
+
+/* Nearest binary16 to x, ties to even; overflow to infinity. */
+uint16_t qo_f64_to_f16(double x)
+{
+    uint16_t sign = signbit(x) ? 0x8000 : 0;
+    double a = fabs(x);
+    if (isnan(x))
+        return 0x7e00;
+    if (a >= 65520.0)                 /* halfway between 65504 and 2^16 rounds up */
+        return sign | 0x7c00;
+    if (a < ldexp(1.0, -14)) {        /* subnormal range: multiples of 2^-24 */
+        double q = nearbyint(ldexp(a, 24));          /* default mode: ties to even */
+        return sign | (uint16_t)q;    /* q == 1024 is the smallest normal, as bits */
+    }
+    int e2;
+    double f = frexp(a, &e2);         /* a = f * 2^e2, f in [0.5, 1) */
+    int e = e2 - 1;                   /* a = (2f) * 2^e, 2f in [1, 2) */
+    double m = nearbyint((2.0 * f - 1.0) * 1024.0);
+    if (m == 1024.0) {
+        m = 0.0;
+        e += 1;
+    }
+    if (e + 15 >= 31)
+        return sign | 0x7c00;
+    return sign | (uint16_t)(((e + 15) << 10) | (int)m);
+}
+
+void qo_f16_to_f64_array(const uint16_t *h, int64_t n, double *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = qo_f16_to_f64(h[i]);
+}
+
+void qo_f64_to_f16_array(const double *x, int64_t n, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = qo_f64_to_f16(x[i]);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Hadamard matrices and the transform.                                       */
+/* ------------------------------------------------------------------------ */
+
+static int is_pow2(int64_t n) { return n >= 1 && (n & (n - 1)) == 0; }
+
+/*
+ * Sylvester construction: H_1 = [1], H_2m = [[H_m, H_m], [H_m, -H_m]].
+ * Writes the n x n matrix row-major.  Returns 0, or -1 if n is not a power
+ * of two.
+ */
+int qo_sylvester(int64_t n, int8_t *H)
+{
+    if (!is_pow2(n))
+        return -1;
+    H[0] = 1;
+    for (int64_t m = 1; m < n; m *= 2) {
+        for (int64_t i = 0; i < m; ++i) {
+            for (int64_t j = 0; j < m; ++j) {
+                int8_t h = H[i * n + j];
+                H[i * n + (j + m)] = h;
+                H[(i + m) * n + j] = h;
+                H[(i + m) * n + (j + m)] = (int8_t)-h;
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * Unnormalized fast Walsh-Hadamard transform in place: v <- v * H_n, Sylvester
+ * order (H_n is symmetric, so this is also H_n * v).  The textbook butterfly:
+ * for each span h = 1, 2, 4, ..., n/2, replace every pair (a, b) that is h
+ * apart inside a block of 2h by (a + b, a - b).
+ */
+int qo_fwht(double *v, int64_t n)
+{
+    if (!is_pow2(n))
+        return -1;
+    for (int64_t h = 1; h < n; h *= 2) {
+        for (int64_t i = 0; i < n; i += 2 * h) {
+            for (int64_t j = i; j < i + h; ++j) {
+                double a = v[j], b = v[j + h];
+                v[j] = a + b;
+                v[j + h] = a - b;
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * The online randomized rotation of the activations (QuaRot summary and
+ * article: randomized Hadamard; DuQuant Knowl 2 and 12: block-diagonal
+ * rotations of block 128).  For each row x of X (fp16 bits, M x K):
+ *     x' = (x * diag(s)) * R,
+ * where R = H_K / sqrt(K) when had_block == 0 (K a power of two), and
+ * R = I_{K/b} (x) (H_b / sqrt(b)) when had_block == b (each b-wide block of
+ * the row rotated on its own).  Output fp64, M x K.
+ */
+int qo_rotate(const uint16_t *x16, int64_t M, int64_t K, const int8_t *signs,
+              int64_t had_block, double *out)
+{
+    int64_t n = had_block == 0 ? K : had_block;
+    if (!is_pow2(n) || K % n != 0 || M < 0)
+        return -1;
+    double inv = 1.0 / sqrt((double)n);
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; ++r) {
+        double *o = out + r * K;
+        for (int64_t k = 0; k < K; ++k)
+            o[k] = qo_f16_to_f64(x16[r * K + k]) * (double)signs[k];
+        for (int64_t b0 = 0; b0 < K; b0 += n) {
+            qo_fwht(o + b0, n);
+            for (int64_t k = 0; k < n; ++k)
+                o[b0 + k] *= inv;
+        }
+    }
+    return 0;
+}
+
+/*
+ * The same rotation as a dense product with the Sylvester matrix:
+ * x'[k] = sum_l x[l] s[l] H[l][k] / sqrt(n), block by block.  O(n^2) per
+ * block; used for small n and as a second route in the tests.
+ */
+int qo_rotate_dense(const uint16_t *x16, int64_t M, int64_t K, const int8_t *signs,
+                    int64_t had_block, double *out)
+{
+    int64_t n = had_block == 0 ? K : had_block;
+    if (!is_pow2(n) || K % n != 0 || M < 0 || n > 8192)
+        return -1;
+    int8_t *H = (int8_t *)malloc((size_t)(n * n));
+    if (!H)
+        return -2;
+    qo_sylvester(n, H);
+    double inv = 1.0 / sqrt((double)n);
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; ++r) {
+        for (int64_t b0 = 0; b0 < K; b0 += n) {
+            for (int64_t k = 0; k < n; ++k) {
+                double acc = 0.0;
+                for (int64_t l = 0; l < n; ++l)
+                    acc += qo_f16_to_f64(x16[r * K + b0 + l]) * (double)signs[b0 + l] *
+                           (double)H[l * n + k];
+                out[r * K + b0 + k] = acc * inv;
+            }
+        }
+    }
+    free(H);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Symmetric round-to-nearest INT4 quantization (QuaRot key points: RTN).      */
+/* ------------------------------------------------------------------------ */
+
+/* q = clamp(rint(v / s), -8, 7); a zero scale gives a zero code. */
+static int8_t rtn_code(double v, double s)
+{
+    if (s == 0.0)
+        return 0;
+    double q = nearbyint(v / s);      /* ties to even */
+    if (q < -8.0)
+        q = -8.0;
+    if (q > 7.0)
+        q = 7.0;
+    return (int8_t)q;
+}
+
+/*
+ * Quantize the rotated values xr (M x K, fp64).
+ *  group == 0:   one scale per row, s = max|row| / 7, kept in fp64 (scale64[M]).
+ *  group == g>0: one scale per (row, g-wide group), s16 = fp16(max|group| / 7)
+ *                stored in scale16[M, K/g]; the codes use the stored fp16 value.
+ * Codes are written unpacked, one int8 per element.
+ */
+int qo_quantize(const double *xr, int64_t M, int64_t K, int64_t group, int8_t *codes,
+                double *scale64, uint16_t *scale16)
+{
+    if (M < 0 || K <= 0 || group < 0 || (group > 0 && K % group != 0))
+        return -1;
+    int64_t G = group == 0 ? 1 : K / group;
+    int64_t w = group == 0 ? K : group;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; ++r) {
+        for (int64_t g = 0; g < G; ++g) {
+            const double *v = xr + r * K + g * w;
+            double amax = 0.0;
+            for (int64_t k = 0; k < w; ++k)
+                if (fabs(v[k]) > amax)
+                    amax = fabs(v[k]);
+            double s;
+            if (group == 0) {
+                s = amax / 7.0;
+                scale64[r] = s;
+            } else {
+                uint16_t h = qo_f64_to_f16(amax / 7.0);
+                scale16[r * G + g] = h;
+                s = qo_f16_to_f64(h);
+            }
+            for (int64_t k = 0; k < w; ++k)
+                codes[r * K + g * w + k] = rtn_code(v[k], s);
+        }
+    }
+    return 0;
+}
+
+/* Nibble packing: byte i = code[2i] in bits 0-3, code[2i+1] in bits 4-7. */
+int qo_pack(const int8_t *codes, int64_t n, uint8_t *packed)
+{
+    if (n % 2 != 0)
+        return -1;
+    for (int64_t i = 0; i < n / 2; ++i)
+        packed[i] = (uint8_t)((codes[2 * i] & 0x0f) | ((codes[2 * i + 1] & 0x0f) << 4));
+    return 0;
+}
+
+/* Inverse of qo_pack: each nibble read as a 4-bit two's-complement number. */
+int qo_unpack(const uint8_t *packed, int64_t n, int8_t *codes)
+{
+    if (n % 2 != 0)
+        return -1;
+    for (int64_t i = 0; i < n / 2; ++i) {
+        int lo = packed[i] & 0x0f, hi = (packed[i] >> 4) & 0x0f;
+        codes[2 * i] = (int8_t)(lo >= 8 ? lo - 16 : lo);
+        codes[2 * i + 1] = (int8_t)(hi >= 8 ? hi - 16 : hi);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Integer matrix product and dequantization (QuaRot: all matrix products in  */
+/* 4 bits, in integers).                                                      */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * acc[m, n, g] = sum over k in group g of qa[m, k] * qw[n, k], int64.
+ * group == 0 means one group spanning all of K (acc is M x N).
+ */
+int qo_int_gemm(const int8_t *qa, const int8_t *qw, int64_t M, int64_t N, int64_t K,
+                int64_t group, int64_t *acc)
+{
+    if (M < 0 || N < 0 || K <= 0 || group < 0 || (group > 0 && K % group != 0))
+        return -1;
+    int64_t G = group == 0 ? 1 : K / group;
+    int64_t w = group == 0 ? K : group;
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            for (int64_t g = 0; g < G; ++g) {
+                int64_t s = 0;
+                for (int64_t k = g * w; k < (g + 1) * w; ++k)
+                    s += (int64_t)qa[m * K + k] * (int64_t)qw[n * K + k];
+                acc[(m * N + n) * G + g] = s;
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * Dequantized output.  group == 0: y[m, n] = acc[m, n] * sa[m] * sw[n].
+ * group > 0 (G groups): y[m, n] = sum_g acc[m, n, g] * sa[m, g] * sw[n, g].
+ * y64 gets the fp64 value, y16 (if not NULL) its nearest fp16.
+ */
+int qo_dequant_linear(const int64_t *acc, int64_t M, int64_t N, int64_t G, const double *sa,
+                      const double *sw, double *y64, uint16_t *y16)
+{
+    if (M < 0 || N < 0 || G <= 0)
+        return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double y = 0.0;
+            for (int64_t g = 0; g < G; ++g)
+                y += (double)acc[(m * N + n) * G + g] * sa[m * G + g] * sw[n * G + g];
+            y64[m * N + n] = y;
+            if (y16)
+                y16[m * N + n] = qo_f64_to_f16(y);
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* INT4 KV cache (QuaRot abstract: the KV cache in 4 bits; DuQuant Knowl 12:  */
+/* fixed Hadamard rotation on the query-key product with per-head quantization). */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * K, V: fp16 [B, T, H, D].  signs: [H, D].  Each key row k[b, t, h, :] becomes
+ * (k * diag(signs[h])) * H_D / sqrt(D); keys and values are then quantized
+ * with one fp16 scale per (b, t, h) over the D channels.  Values are not
+ * rotated.  Codes unpacked, int8 [B, T, H, D]; scales fp16 [B, T, H].
+ */
+int qo_kv_quant(const uint16_t *k16, const uint16_t *v16, int64_t B, int64_t T, int64_t H,
+                int64_t D, const int8_t *signs, int8_t *kcodes, uint16_t *kscale16,
+                int8_t *vcodes, uint16_t *vscale16)
+{
+    if (!is_pow2(D) || B < 0 || T < 0 || H <= 0)
+        return -1;
+    int64_t rows = B * T;
+    int64_t W = H * D;
+    double *tmp = (double *)malloc((size_t)(rows * W) * sizeof(double));
+    if (!tmp && rows > 0)
+        return -2;
+    /* keys: the row of H heads is rotated block-wise, block D, with the
+       concatenated per-head sign vectors; the scale groups are the heads */
+    int rc = qo_rotate(k16, rows, W, signs, D, tmp);
+    if (rc == 0)
+        rc = qo_quantize(tmp, rows, W, D, kcodes, NULL, kscale16);
+    /* values: no rotation */
+    if (rc == 0) {
+        for (int64_t i = 0; i < rows * W; ++i)
+            tmp[i] = qo_f16_to_f64(v16[i]);
+        rc = qo_quantize(tmp, rows, W, D, vcodes, NULL, vscale16);
+    }
+    free(tmp);
+    return rc;
+}
+
+/*
+ * One decode step of query-key scores over the INT4 key cache.
+ * q: fp16 [B, Hq, D]; query head hq uses KV head hq / (Hq / H).
+ * q' = (q * diag(signs[h])) * H_D / sqrt(D), kept in fp64 (not quantized);
+ * scores[b, hq, t] = sum_d q'[d] * kcodes[b, t, h, d] * kscale[b, t, h].
+ */
+int qo_kv_scores(const uint16_t *q16, int64_t B, int64_t Hq, int64_t H, int64_t D, int64_t T,
+                 const int8_t *signs, const int8_t *kcodes, const double *kscale,
+                 double *scores)
+{
+    if (!is_pow2(D) || H <= 0 || Hq % H != 0 || B < 0 || T < 0)
+        return -1;
+    int64_t grp = Hq / H;
+#pragma omp parallel for schedule(static)
+    for (int64_t bh = 0; bh < B * Hq; ++bh) {
+        int64_t b = bh / Hq, hq = bh % Hq, h = hq / grp;
+        double *qr = (double *)malloc((size_t)D * sizeof(double));
+        for (int64_t d = 0; d < D; ++d)
+            qr[d] = qo_f16_to_f64(q16[(b * Hq + hq) * D + d]) * (double)signs[h * D + d];
+        qo_fwht(qr, D);
+        double inv = 1.0 / sqrt((double)D);
+        for (int64_t d = 0; d < D; ++d)
+            qr[d] *= inv;
+        for (int64_t t = 0; t < T; ++t) {
+            const int8_t *kc = kcodes + ((b * T + t) * H + h) * D;
+            double s = 0.0;
+            for (int64_t d = 0; d < D; ++d)
+                s += qr[d] * (double)kc[d];
+            scores[(b * Hq + hq) * T + t] = s * kscale[(b * T + t) * H + h];
+        }
+        free(qr);
+    }
+    return 0;
+}
+
+int qo_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
