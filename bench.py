@@ -1,0 +1,408 @@
+#!/usr/bin/env python
+"""Benchmark of the QuaRot hot path on B200 (one JSON line on rank 0).
+
+One step = every row of the path over one batch of seeded synthetic input:
+  * the LLaMA-2-70B-shaped prefill linear: 32768 tokens x K 8192, online
+    H_8192 randomized rotation + per-token INT4 quantization (quarot_rotate_quant),
+    then the INT4 x INT4 GEMM to N 28672 with the dequantizing epilogue
+    (quarot_int4_linear); the weights are rotated and quantized once, offline;
+  * the 70B GQA INT4 KV cache: write (quarot_kv_quant) of K and V
+    [64, 2048, 8, 128] and one decode step of scores for 64 query heads
+    (quarot_kv_decode_scores).
+value = INT4 linear tera-ops (2 M N K per step, all ranks) / device time of
+the whole step (max over ranks).  Inputs and outputs are larger than L2
+(X 512 MiB, output 1.75 GiB, K/V 256 MiB each), so L2 is not flushed.
+
+--impl reference times the CPU oracle on a bounded sample of the same step
+and extrapolates linearly to the full workload.
+Multi-GPU (torchrun): replicas only -- every rank runs the same step on its
+own GPU, no collective on the data path.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "INT4 linear TOPS + rotate/quant GB/s at 1 B200 (% of roofline)"
+WORKLOAD = ("llama2-70b prefill linear 32768 tok x K 8192 (H_8192, per-token INT4) -> N 28672 fp16, "
+            "+ INT4 KV cache write B64 T2048 Hkv8 D128 and one decode step of 64 q-heads")
+LAUNCHES_PER_STEP = 5            # rotate_quant, int4 GEMM, kv quant (K, V), decode scores
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--cpu-rows", type=int, default=192, help="token rows of the CPU-baseline sample")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sust=d["bf16_tflops_sustained"],
+                    src="of measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, src="of fallback")
+
+
+def source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "rotation_bit_quantization_randomized_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if taken on this source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(kernel)
+    if not e or e.get("source_sha") != source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """NVML samples of SM clock and clock-event reasons while running."""
+    BITS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+            0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle"}
+
+    def __init__(self, index):
+        self.index, self.samples, self.reasons, self.stop_ev = index, [], set(), threading.Event()
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self.stop_ev.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for b, name in self.BITS.items():
+                    if r & b and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.02)
+
+    def __enter__(self):
+        if self.nv:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.nv:
+            self.stop_ev.set()
+            self.t.join()
+
+    def result(self):
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+def bytes_rotate_quant(M, K):
+    return M * K * 2 + M * K // 2 + M * 4
+
+
+def bytes_kv_quant(B, T, H, D):
+    e = B * T * H * D
+    return 2 * (e * 2) + 2 * (e // 2) + 2 * (B * T * H * 2)
+
+
+def bytes_kv_scores(B, T, H, D, Hq):
+    return B * T * H * (D // 2 + 2) + B * Hq * D * 2 + B * Hq * T * 4
+
+
+# ---------------------------------------------------------------------------------------------
+
+def cpu_reference_step(w, c, rows, kv_batches, x, qw_codes, sw, s, kv):
+    """The oracle on a sample of one step; returns (seconds, sample description)."""
+    import oracle
+    t0 = time.perf_counter()
+    qa, sa, _ = oracle.rotate_quant(x[:rows], s, 0, 0)
+    acc = oracle.int_gemm(oracle.unpack(qa), qw_codes, 0)
+    oracle.dequant_linear(acc, sa, sw, 0)
+    t_lin = time.perf_counter() - t0
+    k, v, qh, sk = kv
+    t0 = time.perf_counter()
+    kq, ks, _, _ = oracle.kv_quant(k[:kv_batches], v[:kv_batches], sk)
+    oracle.kv_scores(qh[:kv_batches], sk, kq, ks)
+    t_kv = time.perf_counter() - t0
+    full = t_lin * (w.M / rows) + t_kv * (c.B / kv_batches)
+    desc = (f"{rows} of {w.M} tokens through rotate+quantize+int64 GEMM+dequant against all {w.Ns[0]} "
+            f"channels ({t_lin:.1f} s) and {kv_batches} of {c.B} KV batches through write+decode scores "
+            f"({t_kv:.1f} s); step time scaled linearly to the full workload")
+    return full, desc, t_lin + t_kv
+
+
+def cpu_inputs(w, c, kv_batches):
+    import oracle
+    from rotation_bit_quantization_randomized_b200 import synth
+    s = synth.signs(w.K, w.seed)
+    W = synth.weights(w, w.Ns[0])
+    qw, sw, _ = oracle.rotate_quant(W, s, 0, 0)
+    del W
+    kv = synth.kv_inputs(c, batch=kv_batches)
+    return s, oracle.unpack(qw), sw, kv
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    import oracle
+    from rotation_bit_quantization_randomized_b200 import synth
+    w, c = synth.LLAMA2_70B, synth.KV_70B
+    rows, kvb = 16, 1
+    x = synth.activations(w, rows=max(rows, args.cpu_rows))
+    s, qw_codes, sw, kv = cpu_inputs(w, c, kvb)
+    for _ in range(args.warmup):
+        cpu_reference_step(w, c, rows, kvb, x, qw_codes, sw, s, kv)
+    times, desc = [], ""
+    for _ in range(args.steps):
+        full, desc, _ = cpu_reference_step(w, c, rows, kvb, x, qw_codes, sw, s, kv)
+        times.append(full)
+    t = statistics.mean(times)
+    ops = 2.0 * w.M * w.Ns[0] * w.K
+    value = ops / t / 1e12
+    cores = oracle.max_threads()
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64/int64", "data": "synthetic",
+        "config": {"workload": WORKLOAD},
+        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+# ---------------------------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local_rank, dist):
+    import torch
+    from rotation_bit_quantization_randomized_b200 import binding as q
+    from rotation_bit_quantization_randomized_b200 import synth
+
+    dev = torch.device(f"cuda:{local_rank}")
+    torch.cuda.set_device(dev)
+    w, c = synth.LLAMA2_70B, synth.KV_70B
+    M, K, N = w.M, w.K, w.Ns[0]
+
+    # ---- inputs (seeded synthetic), resident in HBM before timing
+    x_h = synth.activations(w)
+    s_h = synth.signs(K, w.seed)
+    W_h = synth.weights(w, N)
+    k_h, v_h, qh_h, sk_h = synth.kv_inputs(c)
+    x = torch.from_numpy(x_h).to(dev)
+    s = torch.from_numpy(s_h).to(dev)
+    Wd = torch.from_numpy(W_h).to(dev)
+    qw, sw = q.quarot_rotate_quant(Wd, s, 0, 0)          # offline weight preparation
+    del Wd, W_h
+    k = torch.from_numpy(k_h).to(dev)
+    v = torch.from_numpy(v_h).to(dev)
+    qh = torch.from_numpy(qh_h).to(dev)
+    sk = torch.from_numpy(sk_h).to(dev)
+    qa = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+    sa = torch.empty((M,), dtype=torch.float32, device=dev)
+    out = torch.empty((M, N), dtype=torch.float16, device=dev)
+    kq = torch.empty((c.B, c.T, c.Hkv, c.D // 2), dtype=torch.uint8, device=dev)
+    vq = torch.empty_like(kq)
+    ks = torch.empty((c.B, c.T, c.Hkv), dtype=torch.float16, device=dev)
+    vs = torch.empty_like(ks)
+    scores = torch.empty((c.B, c.Hq, c.T), dtype=torch.float32, device=dev)
+
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        q.quarot_rotate_quant(x, s, 0, 0, qa, sa)
+        if ev is not None:
+            ev[1].record(stream)
+        q.quarot_int4_linear(qa, sa, qw, sw, 0, out)
+        if ev is not None:
+            ev[2].record(stream)
+        q.quarot_kv_quant(k, v, sk, kq, ks, vq, vs)
+        if ev is not None:
+            ev[3].record(stream)
+        q.quarot_kv_decode_scores(qh, sk, kq, ks, scores)
+        if ev is not None:
+            ev[4].record(stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if q.quarot_get_device_status() != 0:
+        raise RuntimeError("device status not OK after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    if q.quarot_get_device_status() != 0:
+        raise RuntimeError("device status not OK after the timed region")
+    per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(args.steps)])
+    k_ms = per.mean(axis=0)
+
+    if dist is not None:
+        import torch.distributed as tdist
+        t = torch.tensor([total_ms], device=dev)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    ms_step = total_ms / args.steps
+    ops = 2.0 * M * N * K
+    value = ops * world / (ms_step * 1e-3) / 1e12
+    pk = peaks()
+    int8_sust = 2.0 * pk["bf16_sust"]
+    gemm_tops = ops / (k_ms[1] * 1e-3) / 1e12
+    rq_gbs = bytes_rotate_quant(M, K) / (k_ms[0] * 1e-3) / 1e9
+    kvq_gbs = bytes_kv_quant(c.B, c.T, c.Hkv, c.D) / (k_ms[2] * 1e-3) / 1e9
+    kvs_gbs = bytes_kv_scores(c.B, c.T, c.Hkv, c.D, c.Hq) / (k_ms[3] * 1e-3) / 1e9
+    traffic = recorded_traffic("int4_gemm_kernel")
+
+    # ---- end to end through the public API with host buffers (rank-local)
+    x_p = torch.from_numpy(x_h).pin_memory()
+    k_p = torch.from_numpy(k_h).pin_memory()
+    v_p = torch.from_numpy(v_h).pin_memory()
+    q_p = torch.from_numpy(qh_h).pin_memory()
+    out_p = torch.empty((M, N), dtype=torch.float16).pin_memory()
+    sc_p = torch.empty((c.B, c.Hq, c.T), dtype=torch.float32).pin_memory()
+    ws = torch.empty((q.quarot_rotate_quant_linear_workspace(M, K, 0),), dtype=torch.uint8, device=dev)
+    h2d = sum(t.numel() * t.element_size() for t in (x_p, k_p, v_p, q_p))
+    d2h = out_p.numel() * out_p.element_size() + sc_p.numel() * sc_p.element_size()
+
+    def e2e_step():
+        x.copy_(x_p, non_blocking=True)
+        k.copy_(k_p, non_blocking=True)
+        v.copy_(v_p, non_blocking=True)
+        qh.copy_(q_p, non_blocking=True)
+        q.quarot_rotate_quant_linear(x, s, qw, sw, 0, 0, ws, out)
+        q.quarot_kv_quant(k, v, sk, kq, ks, vq, vs)
+        q.quarot_kv_decode_scores(qh, sk, kq, ks, scores)
+        out_p.copy_(out, non_blocking=True)
+        sc_p.copy_(scores, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    if dist is not None:
+        import torch.distributed as tdist
+        t = torch.tensor([e2e_ms], device=dev)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = ops * world / (e2e_ms * 1e-3) / 1e12
+
+    cpu = None
+    if rank == 0 and world == 1:
+        import oracle
+        rows, kvb = args.cpu_rows, 1
+        s2, qw_codes, sw2, kv = cpu_inputs(w, c, kvb)
+        full_s, desc, spent = cpu_reference_step(w, c, rows, kvb, x_h, qw_codes, sw2, s2, kv)
+        cpu = {"value": ops / full_s / 1e12, "unit": "TOPS", "cores": oracle.max_threads(), "kind": "oracle",
+               "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "i8 (INT4 codes on the int8 tensor path, int32 accumulate; fp32 rotation)",
+            "data": "synthetic (seeded numpy: Student-t3 activations with outlier channels, N(0,0.015) weights, "
+                    "N(0,1) KV with outlier key channels)",
+            "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N, "kv": [c.B, c.T, c.Hkv, c.D], "q_heads": c.Hq,
+                       "l2": "inputs and outputs larger than L2; no explicit flush",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "tensor", "kernel": "int4_gemm_kernel (quarot_int4_linear)",
+                         "achieved": gemm_tops, "peak": int8_sust, "unit": "TFLOP/s",
+                         "frac": gemm_tops / int8_sust, "traffic": traffic,
+                         "peak_note": f"int8 dense = 2 x bf16 sustained {pk['bf16_sust']} {pk['src']}"},
+            "rotate_quant_roofline": {"bound": "hbm", "kernel": "fwht_quant_kernel<13,0> (quarot_rotate_quant)",
+                                      "achieved": rq_gbs, "peak": pk["hbm"], "unit": "GB/s",
+                                      "frac": rq_gbs / pk["hbm"], "traffic": recorded_traffic("fwht_quant_kernel"),
+                                      "peak_note": f"HBM copy {pk['src']}"},
+            "components_ms": {"rotate_quant": k_ms[0], "int4_linear": k_ms[1], "kv_quant": k_ms[2],
+                              "kv_decode_scores": k_ms[3]},
+            "components": {"rotate_quant_gbs": rq_gbs, "int4_linear_tops": gemm_tops, "kv_quant_gbs": kvq_gbs,
+                           "kv_decode_scores_gbs": kvs_gbs},
+            "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "api": "quarot_rotate_quant_linear + quarot_kv_quant + quarot_kv_decode_scores"},
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "clocks": clk.result(),
+            "cpu_baseline": cpu,
+            "source_sha": source_hash(),
+        }
+        print(json.dumps(line))
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(local_rank)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        dist = tdist
+    try:
+        run_ours(args, rank, world, local_rank, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,204 @@
+/*
+ * quarot.h -- C ABI of libquarot, the B200 (sm_100a) hot path of QuaRot
+ * inference: online randomized Hadamard rotation + INT4 round-to-nearest
+ * quantization, INT4 x INT4 linear layers with a dequantizing epilogue, and
+ * an INT4 KV cache with a per-head Hadamard.
+ *
+ * Sources (page title, section):
+ *  [QR-A] QuaRot: Outlier-free 4-bit inference in rotated LLMs -- ISTA research
+ *         explorer record, abstract: weights, activations and KV cache in 4
+ *         bits; rotations leave the output unchanged; all matrix
+ *         multiplications in 4 bits.
+ *  [QR-S] QuaRot: Outlier-Free 4-Bit Inference in Rotated LLMs -- Elamur
+ *         Research summary, "Summary" (random orthogonal Hadamard matrices,
+ *         most fused into the weights, a few applied at inference; products
+ *         in integers) and "Key points" (activations quantized on the fly with
+ *         round-to-nearest; group-wise variant with group size 128).
+ *  [QR-N] QuaRot news article (onlyaistuff.com): randomized Hadamard
+ *         transformations and computational invariance.
+ *  [DQ-1], [DQ-2], [DQ-12] DuQuant (chapterpal) Knowl 1 (Y = XW =
+ *         (XG)(G^-1 W)), Knowl 2 (block-diagonal rotations of 2^n channels),
+ *         Knowl 12 (block size 128; a fixed +-1/sqrt(2^n) Hadamard on the
+ *         query-key product with per-head quantization).
+ *
+ * Conventions for every entry point:
+ *  - All array pointers are DEVICE memory owned by the caller; the library
+ *    allocates nothing (except where an entry point says otherwise) and keeps
+ *    no state beyond a per-device cache of kernel attributes.
+ *  - Every array pointer must be 16-byte aligned; arrays are dense row-major.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream).  Argument errors are returned before any launch and
+ *    leave every output untouched.  A launch failure returns
+ *    QUAROT_ERR_CUDA; quarot_last_error() then gives the CUDA message.
+ *  - fp16 is IEEE binary16.  INT4 codes are two's complement in [-8, 7],
+ *    packed two per byte: element 2i in bits 0-3, element 2i+1 in bits 4-7.
+ *  - No function throws; none blocks the host except
+ *    quarot_get_device_status().
+ */
+#ifndef QUAROT_H
+#define QUAROT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QUAROT_OK = 0,
+    QUAROT_ERR_INVALID_ARG = 1,      /* null pointer, negative size, bad enum value */
+    QUAROT_ERR_UNSUPPORTED_SHAPE = 2,/* a size outside the limits stated per call */
+    QUAROT_ERR_MISALIGNED = 3,       /* a pointer not 16-byte aligned */
+    QUAROT_ERR_CUDA = 4,             /* the CUDA runtime reported an error */
+    QUAROT_ERR_DEVICE_TIMEOUT = 5,   /* a kernel gave up a bounded wait (see below) */
+    QUAROT_ERR_NO_DEVICE = 6         /* no sm_100 device is current */
+} quarot_status_t;
+
+/* A cudaStream_t passed as an opaque pointer. */
+typedef void *quarot_stream_t;
+
+/*
+ * quarot_rotate_quant -- online rotation + INT4 RTN quantization + packing
+ * of activations [QR-S Summary, Key points; QR-N; DQ-2; DQ-12].
+ *
+ *   x'  = (x * diag(signs)) * R,  R = H_K / sqrt(K)              (had_block == 0)
+ *                                 R = I_{K/128} (x) H_128/sqrt(128) (had_block == 128)
+ *   H is the Sylvester-ordered Hadamard matrix.
+ *   group == 0:   s[m] = max_k |x'[m,k]| / 7, stored fp32;  q = rint(x'/s)
+ *   group == 128: s[m,g] = fp16(max over the 128-group |x'| / 7); q = clamp(rint(x'/s16), -8, 7)
+ *   (round half to even; a zero stored scale gives zero codes.)
+ * The rotated values are kept in fp32 inside the kernel and never stored.
+ * The same call prepares weights offline (rows of W are rows of x; group 0
+ * then gives one fp32 scale per output channel) [QR-S Summary].
+ *
+ * x_f16     [M, K] fp16, read only.
+ * signs     [K] int8, each +1 or -1 (any negative value counts as -1).
+ * had_block 0 (K a power of two, 128 <= K <= 8192) or 128 (K % 128 == 0,
+ *           128 <= K <= 65536).
+ * group     0 or 128.
+ * q_packed  [M, K/2] uint8 output.
+ * scales    group 0: fp32 [M]; group 128: fp16 [M, K/128].  Output.
+ * M         >= 0; M == 0 launches nothing and returns QUAROT_OK.
+ */
+quarot_status_t quarot_rotate_quant(const void *x_f16, int64_t M, int64_t K,
+                                    const int8_t *signs, int had_block, int group,
+                                    uint8_t *q_packed, void *scales, quarot_stream_t stream);
+
+/*
+ * quarot_int4_linear -- INT4 x INT4 linear layer with int32 accumulation on
+ * the tensor cores and a fused dequantizing epilogue [QR-A: all matrix
+ * multiplications in 4 bits; QR-S Summary: integer products].
+ *
+ *   group == 0:   out[m,n] = fp16( acc[m,n] * s_a[m] * s_w[n] ),
+ *                 acc[m,n] = sum_k qa[m,k] * qw[n,k]  (int32, exact)
+ *   group == 128: out[m,n] = fp16( sum_g acc_g[m,n] * s_a[m,g] * s_w[n,g] ),
+ *                 acc_g over k in [128g, 128g+128), sum in fp32
+ *
+ * qa   [M, K/2] packed INT4 activations (from quarot_rotate_quant).
+ * s_a  group 0: fp32 [M]; group 128: fp16 [M, K/128].
+ * qw   [N, K/2] packed INT4 weights, the rows rotated with the same signs and
+ *      Hadamard as the activations (computational invariance [DQ-1]).
+ * s_w  group 0: fp32 [N]; group 128: fp16 [N, K/128].
+ * out  [M, N] fp16 output.
+ * Limits: M >= 0 (0 launches nothing), N >= 1 with N % 8 == 0,
+ *         K % 128 == 0 with 128 <= K <= 65536.
+ */
+quarot_status_t quarot_int4_linear(const uint8_t *qa, const void *s_a, int64_t M,
+                                   const uint8_t *qw, const void *s_w, int64_t N, int64_t K,
+                                   int group, void *out_f16, quarot_stream_t stream);
+
+/*
+ * quarot_int4_gemm_s32 -- the same integer product without the epilogue:
+ * acc[m,n] = sum_k qa[m,k] * qw[n,k] written as int32 [M, N].  Exact for
+ * every input (|acc| <= 64 K).  Same layouts and limits as
+ * quarot_int4_linear (no scales).  For testing the integer path in
+ * isolation [QR-S Summary: matrix multiplications in integers].
+ */
+quarot_status_t quarot_int4_gemm_s32(const uint8_t *qa, int64_t M, const uint8_t *qw,
+                                     int64_t N, int64_t K, int32_t *acc,
+                                     quarot_stream_t stream);
+
+/*
+ * quarot_rotate_quant_linear_workspace -- bytes of device workspace that
+ * quarot_rotate_quant_linear needs for M tokens of K channels: the packed
+ * INT4 activations and their scales, each at a 256-byte aligned offset.
+ */
+size_t quarot_rotate_quant_linear_workspace(int64_t M, int64_t K, int group);
+
+/*
+ * quarot_rotate_quant_linear -- the fused online path of one linear layer:
+ * quarot_rotate_quant of x into `workspace`, then quarot_int4_linear against
+ * the prepared weights, both on `stream`; the GEMM is launched as a
+ * programmatic dependent of the quantizer so that its set-up overlaps the
+ * quantizer's tail [QR-S Summary: a few rotations are performed online].
+ *
+ * Arguments as in the two calls above.  workspace: caller-owned device
+ * memory of at least quarot_rotate_quant_linear_workspace(M, K, group) bytes,
+ * 256-byte aligned; its contents are scratch (overwritten, no meaning after
+ * the call).  ws_bytes: its size.
+ */
+quarot_status_t quarot_rotate_quant_linear(const void *x_f16, int64_t M, int64_t K,
+                                           const int8_t *signs, int had_block, int group,
+                                           const uint8_t *qw, const void *s_w, int64_t N,
+                                           void *workspace, size_t ws_bytes, void *out_f16,
+                                           quarot_stream_t stream);
+
+/*
+ * quarot_kv_quant -- INT4 KV-cache write [QR-A: the KV cache in 4 bits;
+ * DQ-12: fixed Hadamard on the query-key product, per-head quantization].
+ *
+ *   key row k[b,t,h,:]:   k' = (k * diag(signs[h,:])) * H_D / sqrt(D), then
+ *                         s = fp16(max|k'| / 7), q = clamp(rint(k'/s), -8, 7)
+ *   value row v[b,t,h,:]: not rotated; same quantizer.
+ *
+ * k_f16, v_f16  [B, T, Hkv, D] fp16.       signs [Hkv, D] int8 (+-1).
+ * kq, vq        [B, T, Hkv, D/2] uint8 packed codes (outputs).
+ * ks_f16, vs_f16 [B, T, Hkv] fp16 scales (outputs).
+ * Limits: D == 128; B, T >= 0; 1 <= Hkv <= 512.
+ */
+quarot_status_t quarot_kv_quant(const void *k_f16, const void *v_f16, int64_t B, int64_t T,
+                                int64_t Hkv, int64_t D, const int8_t *signs, uint8_t *kq,
+                                void *ks_f16, uint8_t *vq, void *vs_f16,
+                                quarot_stream_t stream);
+
+/*
+ * quarot_kv_decode_scores -- one decode step of query-key scores against the
+ * INT4 key cache [QR-A: aspects of the attention mechanism; DQ-12].
+ *
+ *   q'[b,hq,:] = (q[b,hq,:] * diag(signs[h,:])) * H_D / sqrt(D), fp32 (not
+ *                quantized), h = hq / (Hq / Hkv)   (grouped-query attention)
+ *   scores[b,hq,t] = sum_d q'[d] * kq[b,t,h,d] * ks[b,t,h]   (fp32; no 1/sqrt(D),
+ *                no softmax)
+ *
+ * q_f16   [B, Hq, D] fp16.   signs [Hkv, D] int8.
+ * kq      [B, T, Hkv, D/2] packed codes, ks_f16 [B, T, Hkv] fp16 (from quarot_kv_quant).
+ * scores  [B, Hq, T] fp32 output.
+ * Limits: D == 128; Hq % Hkv == 0 with Hq / Hkv <= 16; B, T >= 0.
+ */
+quarot_status_t quarot_kv_decode_scores(const void *q_f16, int64_t B, int64_t Hq,
+                                        const int8_t *signs, const uint8_t *kq,
+                                        const void *ks_f16, int64_t T, int64_t Hkv, int64_t D,
+                                        float *scores, quarot_stream_t stream);
+
+/*
+ * quarot_get_device_status -- synchronizes the current device, then reports
+ * (and clears) the library's device-side error word: QUAROT_ERR_DEVICE_TIMEOUT
+ * if any kernel since the last call gave up a bounded wait (every wait inside
+ * the tensor-core GEMM is bounded in time; on expiry the kernel records the
+ * fact, drains its own in-flight work, frees its tensor memory and exits),
+ * QUAROT_ERR_CUDA if the synchronization itself failed, else QUAROT_OK.
+ */
+quarot_status_t quarot_get_device_status(void);
+
+/* Static, human-readable name of a status code. */
+const char *quarot_status_string(quarot_status_t status);
+
+/* Message of the last QUAROT_ERR_CUDA / argument error on this host thread. */
+const char *quarot_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QUAROT_H */

@@ -40,6 +40,7 @@ def lib():
             "qo_rotate": [P, I64, I64, P, I64, P],
             "qo_rotate_dense": [P, I64, I64, P, I64, P],
             "qo_quantize": [P, I64, I64, I64, P, P, P],
+            "qo_quantize_with_scales": [P, I64, I64, I64, P, P],
             "qo_pack": [P, I64, P],
             "qo_unpack": [P, I64, P],
             "qo_int_gemm": [P, P, I64, I64, I64, I64, P],
@@ -146,6 +147,16 @@ def quantize(xr, group: int = 0):
         sc = np.empty((M, K // group), np.uint16)
         _check(lib().qo_quantize(_p(xr), M, K, group, _p(codes), None, _p(sc)), "quantize")
     return codes, sc
+
+
+def quantize_with_scales(xr, scales, group: int = 0) -> np.ndarray:
+    """RTN codes of xr [M, K] under given scales (fp64 [M], or fp16 bits [M, K/group])."""
+    xr = _c(xr, np.float64)
+    M, K = xr.shape
+    sc = _c(scales_to_f64(scales), np.float64)
+    codes = np.empty((M, K), np.int8)
+    _check(lib().qo_quantize_with_scales(_p(xr), M, K, group, _p(sc), _p(codes)), "quantize_with_scales")
+    return codes
 
 
 def pack(codes) -> np.ndarray:

@@ -277,6 +277,26 @@ int qo_quantize(const double *xr, int64_t M, int64_t K, int64_t group, int8_t *c
     return 0;
 }
 
+/*
+ * The RTN step alone with scales supplied by the caller (one per row when
+ * group == 0, else one per group): q = clamp(rint(v/s), -8, 7), zero scale ->
+ * zero code.  Used to state the expected codes once a scale has been checked.
+ */
+int qo_quantize_with_scales(const double *xr, int64_t M, int64_t K, int64_t group,
+                            const double *scales, int8_t *codes)
+{
+    if (M < 0 || K <= 0 || group < 0 || (group > 0 && K % group != 0))
+        return -1;
+    int64_t G = group == 0 ? 1 : K / group;
+    int64_t w = group == 0 ? K : group;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; ++r)
+        for (int64_t g = 0; g < G; ++g)
+            for (int64_t k = 0; k < w; ++k)
+                codes[r * K + g * w + k] = rtn_code(xr[r * K + g * w + k], scales[r * G + g]);
+    return 0;
+}
+
 /* Nibble packing: byte i = code[2i] in bits 0-3, code[2i+1] in bits 4-7. */
 int qo_pack(const int8_t *codes, int64_t n, uint8_t *packed)
 {

@@ -1,0 +1,439 @@
+// int4_gemm.cuh -- INT4 x INT4 linear layer on the sm_100a tensor cores.
+//
+// QuaRot abstract (ISTA record): all matrix multiplications run in 4 bits;
+// QuaRot summary: products in integers.  The tensor cores have no 4-bit
+// integer kind, so packed nibbles are widened to 8-bit and multiplied with
+// tcgen05.mma.kind::i8 (int32 accumulation in tensor memory); |code| <= 8, so
+// the int32 sums are exact.
+//
+//   acc[m, n]  = sum_k qa[m, k] qw[n, k]
+//   out[m, n]  = fp16(acc * s_a[m] * s_w[n])                       (per token / channel)
+//   out[m, n]  = fp16(sum_g acc_g[m, n] * s_a[m, g] * s_w[n, g])   (groups of 128)
+//
+// Kernel structure (persistent, one CTA per SM, warp-specialized):
+//  * loader warps (each thread owns two tile rows of A or B): read 64 packed
+//    bytes of each row per 128-wide K block straight from global memory
+//    (prefetched two blocks ahead into registers), widen each nibble to
+//    an int8 equal to 16 * code (the nibble lands in the top half of its
+//    byte, so the sign comes for free), and store them into a 4-stage ring in
+//    the 128-byte-swizzled K-major layout the tensor core reads.  Inside each
+//    32-wide K chunk the widened order is [low nibbles, high nibbles]; A and B
+//    use the same order, so every dot product is unchanged.  Both operands
+//    are scaled by 16, so the accumulator holds 256 * acc, removed exactly in
+//    the epilogue (|256 acc| <= 2^14 K < 2^31 for K <= 65536).
+//  * one MMA thread: waits for a full stage, issues four 128 x BN x 32
+//    tcgen05.mma, and commits to the stage's "empty" barrier; at the end of a
+//    tile it commits to the accumulator's "full" barrier.  Two accumulator
+//    buffers in tensor memory let the epilogue of tile i overlap the
+//    mainloop of tile i+1.
+//  * epilogue warps: tcgen05.ld the accumulator (warp w reads TMEM lanes
+//    32(w%4)..+31 = tile rows), scale, convert, store.
+//  * every wait is bounded in time; on expiry the CTA records a timeout in
+//    the device status word, drains its issued MMAs and frees tensor memory.
+#pragma once
+
+#include "common.cuh"
+#include "tc_ptx.cuh"
+
+namespace quarot {
+
+enum : int { kEpiScaledF16 = 0, kEpiS32 = 1, kEpiGroupF16 = 2 };
+
+constexpr int kGemmBM = 128;
+constexpr int kGemmBK = 128;            // int8 elements of K per stage (one 128-byte row)
+constexpr int kGemmStages = 4;
+constexpr int kGemmPrefetch = 2;        // K blocks a loader has in flight ahead of its stores
+constexpr int kGemmGroupM = 16;         // tiles along M that share a band of N tiles
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+template <int BN, int EPI>
+struct GemmShape {
+    static constexpr int kABytes = kGemmBM * kGemmBK;
+    static constexpr int kBBytes = BN * kGemmBK;
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kLoadRows = kGemmBM + BN;      // A rows then B rows of a tile
+    static constexpr int kLoadThreads = kLoadRows / 2;  // two rows per loader thread
+    static constexpr int kEpiWarps = EPI == kEpiGroupF16 ? 8 : 4;
+    static constexpr int kEpiThreads = 32 * kEpiWarps;
+    static constexpr int kMmaWarp = kEpiWarps;
+    static constexpr int kLoadWarp0 = kEpiWarps + 1;
+    static constexpr int kThreads = 32 * (kEpiWarps + 1) + kLoadThreads;
+    static constexpr int kTmemCols = 2 * BN;
+    static constexpr int kBarOffset = kGemmStages * kStageBytes;
+    static constexpr int kNumBars = 2 * kGemmStages + 7;
+    static constexpr int kMiscOffset = kBarOffset + 8 * kNumBars;
+    static constexpr int kSwOffset = kMiscOffset + 16;
+    static constexpr int kSmemBytes = kSwOffset + 2 * BN * 4 + 1024;
+    static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
+    static_assert(kTmemCols == 256 || kTmemCols == 512, "TMEM allocation is a power of two");
+};
+
+struct GemmArgs {
+    const uint8_t *qa;      // [M, K/2]
+    const void *sa;         // fp32 [M] or fp16 [M, K/128]
+    const uint8_t *qw;      // [N, K/2]
+    const void *sw;         // fp32 [N] or fp16 [N, K/128]
+    void *out;              // fp16 or int32 [M, N]
+    int64_t M, N, K;
+    int tiles_m, tiles_n, kblocks;
+};
+
+// Grouped raster: consecutive tile indices walk down kGemmGroupM M-tiles
+// before moving to the next N-tile, so the CTAs working at one time share a
+// small band of A and of W in L2.
+__device__ __forceinline__ void gemm_tile_coords(int t, int tiles_m, int tiles_n, int &mb, int &nb)
+{
+    const int group = kGemmGroupM * tiles_n;
+    const int g = t / group;
+    const int first = g * kGemmGroupM;
+    const int gm = min(kGemmGroupM, tiles_m - first);
+    const int r = t - g * group;
+    mb = first + r % gm;
+    nb = r / gm;
+}
+
+// Bounded wait: true when the phase completed; false when another role gave
+// up (abort flag) or the time limit expired (then this thread sets both).
+__device__ __forceinline__ bool gemm_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity))
+            return true;
+        if (*abort_flag)
+            return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            record_timeout();
+            return false;
+        }
+    }
+}
+
+// Bounded wait that ignores the abort flag (used to drain issued MMAs).
+__device__ __forceinline__ bool gemm_wait_drain(uint32_t bar, uint32_t parity)
+{
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            record_timeout();
+            return false;
+        }
+    }
+    return true;
+}
+
+__device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
+
+// int32 with |v| < 2^22 to float exactly, without the slow conversion unit.
+__device__ __forceinline__ float small_i2f(uint32_t v)
+{
+    return __uint_as_float(v + 0x4B400000u) - 12582912.0f;
+}
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(GemmShape<BN, EPI>::kThreads, 1)
+int4_gemm_kernel(const GemmArgs a)
+{
+    using S = GemmShape<BN, EPI>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar_full = sbase + S::kBarOffset;
+    const uint32_t bar_empty = bar_full + 8 * kGemmStages;
+    const uint32_t bar_accf = bar_empty + 8 * kGemmStages;
+    const uint32_t bar_acce = bar_accf + 16;
+    const uint32_t bar_drain = bar_acce + 16;
+    const uint32_t bar_sws = bar_drain + 8;        // grouped: column-scale staging, 2 buffers
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + S::kMiscOffset);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + S::kMiscOffset + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int num_tiles = a.tiles_m * a.tiles_n;
+    const int KB = a.kblocks;
+    const int my_tiles = blockIdx.x < num_tiles ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kGemmStages; ++s) {
+            mbar_init(bar_full + 8 * s, S::kLoadThreads);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_accf + 8 * b, 1);
+            mbar_init(bar_acce + 8 * b, S::kEpiThreads);
+        }
+        mbar_init(bar_drain, 1);
+        mbar_init(bar_sws, S::kEpiThreads);
+        mbar_init(bar_sws + 8, S::kEpiThreads);
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == S::kMmaWarp) {
+        tmem_alloc(smem_u32(tmem_slot), S::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    // inputs may come from the kernel launched just before (programmatic
+    // dependent launch); everything above overlapped its tail
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    if (warp >= S::kLoadWarp0) {
+        // ------------------------------------------------------------ loaders
+        // thread l owns rows l and l + kLoadThreads of the combined
+        // [A rows 0..127 | B rows 0..BN-1] index space
+        const int l = threadIdx.x - 32 * S::kLoadWarp0;
+        const int64_t ldb = a.K / 2;
+        const int total = my_tiles * KB;
+        int rrow[2];
+        bool isA[2];
+        uint32_t row_off[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int c = l + h * S::kLoadThreads;
+            isA[h] = c < kGemmBM;
+            rrow[h] = isA[h] ? c : c - kGemmBM;
+            row_off[h] = (isA[h] ? 0u : (uint32_t)S::kABytes) + (rrow[h] >> 3) * 1024 + (rrow[h] & 7) * 128;
+        }
+
+        auto fetch = [&](uint4 (&d)[2][4], int step) {
+            const int lt = step / KB;
+            const int kb = step - lt * KB;
+            int mb, nb;
+            gemm_tile_coords(blockIdx.x + lt * gridDim.x, a.tiles_m, a.tiles_n, mb, nb);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int64_t row = (int64_t)(isA[h] ? mb * kGemmBM : nb * BN) + rrow[h];
+                const bool ok = row < (isA[h] ? a.M : a.N);
+                const uint4 *p = reinterpret_cast<const uint4 *>((isA[h] ? a.qa : a.qw) + (ok ? row : 0) * ldb +
+                                                                 (int64_t)kb * 64);
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    d[h][c] = ok ? __ldg(p + c) : make_uint4(0, 0, 0, 0);
+            }
+        };
+
+        uint4 pf[kGemmPrefetch][2][4];
+#pragma unroll
+        for (int p = 0; p < kGemmPrefetch; ++p)
+            if (p < total)
+                fetch(pf[p], p);
+
+        bool ok = true;
+        static_assert(kGemmStages % kGemmPrefetch == 0, "unrolled ring indexing");
+        for (int it = 0; it < total && ok; it += kGemmStages) {
+#pragma unroll
+            for (int p = 0; p < kGemmStages; ++p) {
+                const int step = it + p;          // stage index == p
+                const int slot = p % kGemmPrefetch;
+                if (step < total && ok) {
+                    const uint32_t use = (uint32_t)(step / kGemmStages);
+                    if (!gemm_wait(bar_empty + 8 * p, (use & 1) ^ 1, abort_flag)) {
+                        ok = false;
+                    } else {
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            uint8_t *dst = smem + p * S::kStageBytes + row_off[h];
+                            const int sw = rrow[h] & 7;
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) {
+                                const uint4 w = pf[slot][h][c];
+                                const uint4 lo = make_uint4((w.x << 4) & 0xF0F0F0F0u, (w.y << 4) & 0xF0F0F0F0u,
+                                                            (w.z << 4) & 0xF0F0F0F0u, (w.w << 4) & 0xF0F0F0F0u);
+                                const uint4 hi = make_uint4(w.x & 0xF0F0F0F0u, w.y & 0xF0F0F0F0u,
+                                                            w.z & 0xF0F0F0F0u, w.w & 0xF0F0F0F0u);
+                                *reinterpret_cast<uint4 *>(dst + (((2 * c) ^ sw) << 4)) = lo;
+                                *reinterpret_cast<uint4 *>(dst + (((2 * c + 1) ^ sw) << 4)) = hi;
+                            }
+                        }
+                        fence_proxy_async_smem();
+                        mbar_arrive(bar_full + 8 * p);
+                        if (step + kGemmPrefetch < total)
+                            fetch(pf[slot], step + kGemmPrefetch);
+                    }
+                }
+            }
+        }
+    } else if (warp == S::kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_i8(kGemmBM, BN);
+            bool ok = true;
+            int step = 0;
+            for (int lt = 0; lt < my_tiles && ok; ++lt) {
+                for (int kb = 0; kb < KB && ok; ++kb, ++step) {
+                    const int ab = EPI == kEpiGroupF16 ? (step & 1) : (lt & 1);
+                    const uint32_t ause = EPI == kEpiGroupF16 ? (uint32_t)(step >> 1) : (uint32_t)(lt >> 1);
+                    if (EPI == kEpiGroupF16 || kb == 0) {
+                        if (!gemm_wait(bar_acce + 8 * ab, (ause & 1) ^ 1, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                    }
+                    const int stage = step % kGemmStages;
+                    const uint32_t use = (uint32_t)(step / kGemmStages);
+                    if (!gemm_wait(bar_full + 8 * stage, use & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t as = sbase + stage * S::kStageBytes;
+                    const uint32_t bs = as + S::kABytes;
+                    const uint32_t d = tmem_base + ab * BN;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint32_t acc = (EPI == kEpiGroupF16) ? (j > 0) : (kb > 0 || j > 0);
+                        umma_i8_ss(d, desc_kmajor_sw128(as + 32 * j), desc_kmajor_sw128(bs + 32 * j), idesc, acc);
+                    }
+                    umma_commit(bar_empty + 8 * stage);
+                    if (EPI == kEpiGroupF16 || kb == KB - 1)
+                        umma_commit(bar_accf + 8 * ab);
+                }
+            }
+            umma_commit(bar_drain);
+            gemm_wait_drain(bar_drain, 0);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int wq = warp & 3;                 // TMEM lane quarter of this warp
+        const uint32_t lane_addr = tmem_base + ((uint32_t)(32 * wq) << 16);
+        bool ok = true;
+        int step = 0;
+        for (int lt = 0; lt < my_tiles && ok; ++lt) {
+            int mb, nb;
+            gemm_tile_coords(blockIdx.x + lt * gridDim.x, a.tiles_m, a.tiles_n, mb, nb);
+            const int64_t m = (int64_t)mb * kGemmBM + 32 * wq + lane;
+            const int64_t n0 = (int64_t)nb * BN;
+            const bool mrow = m < a.M;
+
+            if (EPI != kEpiGroupF16) {
+                const int ab = lt & 1;
+                if (!gemm_wait(bar_accf + 8 * ab, (uint32_t)(lt >> 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                float sam = 0.f;
+                if (EPI == kEpiScaledF16 && mrow)
+                    sam = reinterpret_cast<const float *>(a.sa)[m] * (1.0f / 256.0f);
+#pragma unroll 1
+                for (int c = 0; c < BN / 32; ++c) {
+                    uint32_t r[32];
+                    __syncwarp();
+                    tmem_ld32(lane_addr + ab * BN + 32 * c, r);
+                    tmem_wait_ld(r);
+                    if (c == BN / 32 - 1) {
+                        tc_fence_before();
+                        mbar_arrive(bar_acce + 8 * ab);
+                    }
+                    if (mrow && EPI == kEpiScaledF16) {
+                        __half *orow = reinterpret_cast<__half *>(a.out) + m * a.N;
+                        const float *swp = reinterpret_cast<const float *>(a.sw);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            const int64_t n = n0 + 32 * c + 8 * v;
+                            if (n < a.N) {
+                                const float4 w0 = __ldg(reinterpret_cast<const float4 *>(swp + n));
+                                const float4 w1 = __ldg(reinterpret_cast<const float4 *>(swp + n + 4));
+                                const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                                uint32_t h[4];
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) {
+                                    const float f0 = __int2float_rn((int)r[8 * v + 2 * i]) * sam * wv[2 * i];
+                                    const float f1 = __int2float_rn((int)r[8 * v + 2 * i + 1]) * sam * wv[2 * i + 1];
+                                    h[i] = h2_as_u32(__floats2half2_rn(f0, f1));
+                                }
+                                *reinterpret_cast<uint4 *>(orow + n) = make_uint4(h[0], h[1], h[2], h[3]);
+                            }
+                        }
+                    } else if (mrow) {
+                        int32_t *orow = reinterpret_cast<int32_t *>(a.out) + m * a.N;
+#pragma unroll
+                        for (int v = 0; v < 8; ++v) {
+                            const int64_t n = n0 + 32 * c + 4 * v;
+                            if (n < a.N)
+                                *reinterpret_cast<int4 *>(orow + n) =
+                                    make_int4((int)r[4 * v] >> 8, (int)r[4 * v + 1] >> 8,
+                                              (int)r[4 * v + 2] >> 8, (int)r[4 * v + 3] >> 8);
+                        }
+                    }
+                }
+            } else {
+                // grouped: warps w and w+4 share TMEM lanes and split the columns
+                constexpr int HALF = BN / 2;
+                const int col0 = (warp >> 2) * HALF;
+                const int et = threadIdx.x;                      // 0 .. kEpiThreads-1
+                const int G = KB;
+                float accv[HALF];
+#pragma unroll
+                for (int i = 0; i < HALF; ++i)
+                    accv[i] = 0.f;
+                for (int kb = 0; kb < KB; ++kb, ++step) {
+                    const int ab = step & 1;
+                    float *sws = reinterpret_cast<float *>(smem + S::kSwOffset) + ab * BN;
+                    if (et < BN) {
+                        const int64_t n = n0 + et;
+                        sws[et] = n < a.N ? __half2float(reinterpret_cast<const __half *>(a.sw)[n * G + kb]) : 0.f;
+                    }
+                    mbar_arrive(bar_sws + 8 * ab);
+                    if (!gemm_wait(bar_sws + 8 * ab, (uint32_t)(step >> 1) & 1, abort_flag) ||
+                        !gemm_wait(bar_accf + 8 * ab, (uint32_t)(step >> 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const float sag = mrow ? __half2float(reinterpret_cast<const __half *>(a.sa)[m * G + kb]) *
+                                                 (1.0f / 256.0f)
+                                           : 0.f;
+#pragma unroll
+                    for (int c = 0; c < HALF / 16; ++c) {
+                        uint32_t r[16];
+                        __syncwarp();
+                        tmem_ld16(lane_addr + ab * BN + col0 + 16 * c, r);
+                        tmem_wait_ld16(r);
+                        if (c == HALF / 16 - 1) {
+                            tc_fence_before();
+                            mbar_arrive(bar_acce + 8 * ab);
+                        }
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            accv[16 * c + i] = fmaf(small_i2f(r[i]) * sag, sws[col0 + 16 * c + i], accv[16 * c + i]);
+                    }
+                }
+                if (!ok)
+                    break;
+                if (mrow) {
+                    __half *orow = reinterpret_cast<__half *>(a.out) + m * a.N;
+#pragma unroll
+                    for (int v = 0; v < HALF / 8; ++v) {
+                        const int64_t n = n0 + col0 + 8 * v;
+                        if (n < a.N) {
+                            uint32_t h[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                h[i] = h2_as_u32(__floats2half2_rn(accv[8 * v + 2 * i], accv[8 * v + 2 * i + 1]));
+                            *reinterpret_cast<uint4 *>(orow + n) = make_uint4(h[0], h[1], h[2], h[3]);
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == S::kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, S::kTmemCols);
+    }
+}
+
+}  // namespace quarot

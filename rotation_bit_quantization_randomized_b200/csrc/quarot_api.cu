@@ -1,0 +1,480 @@
+// quarot_api.cu -- the C ABI of libquarot (declared in include/quarot.h):
+// argument validation, launch configuration and error reporting around the
+// kernels in rotate_quant.cuh, int4_gemm.cuh and kv_scores.cuh.
+#include "quarot.h"
+
+#include "common.cuh"
+#include "int4_gemm.cuh"
+#include "kv_scores.cuh"
+#include "rotate_quant.cuh"
+
+#include <cmath>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+using namespace quarot;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+quarot_status_t fail(quarot_status_t s, const std::string &msg)
+{
+    g_last_error = msg;
+    return s;
+}
+
+quarot_status_t cuda_fail(cudaError_t e, const char *what)
+{
+    return fail(QUAROT_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+// Per-device facts and one-time kernel attributes.
+struct DeviceInfo {
+    bool init = false;
+    bool ok = false;
+    int sm_count = 0;
+};
+constexpr int kMaxDevices = 64;
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_mutex;
+
+quarot_status_t current_device(int &dev, DeviceInfo *&info)
+{
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices)
+        return fail(QUAROT_ERR_NO_DEVICE, "device ordinal out of range");
+    std::lock_guard<std::mutex> lk(g_mutex);
+    DeviceInfo &d = g_devices[dev];
+    if (!d.init) {
+        int major = 0, minor = 0;
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);
+        d.ok = (major == 10 && minor == 0);
+        d.init = true;
+    }
+    info = &d;
+    if (!d.ok)
+        return fail(QUAROT_ERR_NO_DEVICE, "libquarot needs an sm_100 (B200) device");
+    return QUAROT_OK;
+}
+
+// Resident CTAs per SM of `kernel`, computed once per (kernel, device); also
+// raises the dynamic shared-memory limit when the kernel needs it.
+template <typename K>
+quarot_status_t kernel_occupancy(K kernel, int dev, int threads, size_t dyn_smem, int &per_sm)
+{
+    struct Entry {
+        const void *fn;
+        int dev;
+        int threads;
+        int per_sm;
+    };
+    static Entry cache[256];
+    static int n = 0;
+    std::lock_guard<std::mutex> lk(g_mutex);
+    for (int i = 0; i < n; ++i)
+        if (cache[i].fn == (const void *)kernel && cache[i].dev == dev && cache[i].threads == threads) {
+            per_sm = cache[i].per_sm;
+            return QUAROT_OK;
+        }
+    cudaError_t e;
+    if (dyn_smem > 48 * 1024) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn_smem);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cudaFuncSetAttribute");
+    }
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, dyn_smem);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    if (per_sm < 1)
+        return fail(QUAROT_ERR_CUDA, "kernel does not fit on an SM");
+    if (n < 256)
+        cache[n++] = Entry{(const void *)kernel, dev, threads, per_sm};
+    return QUAROT_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
+
+int ilog2(int64_t v)
+{
+    int l = 0;
+    while ((int64_t(1) << l) < v)
+        ++l;
+    return l;
+}
+
+quarot_status_t after_launch(const char *what)
+{
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return cuda_fail(e, what);
+    return QUAROT_OK;
+}
+
+// ----------------------------------------------------------------- rotate + quantize
+quarot_status_t check_rotate_args(const void *x, int64_t M, int64_t K, const int8_t *signs, int had_block,
+                                  int group, const void *q, const void *scales)
+{
+    if (M < 0 || K <= 0)
+        return fail(QUAROT_ERR_INVALID_ARG, "M must be >= 0 and K > 0");
+    if (had_block != 0 && had_block != 128)
+        return fail(QUAROT_ERR_INVALID_ARG, "had_block must be 0 or 128");
+    if (group != 0 && group != 128)
+        return fail(QUAROT_ERR_INVALID_ARG, "group must be 0 or 128");
+    if (had_block == 0 && (!is_pow2(K) || K < 128 || K > 8192))
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "full Hadamard needs K a power of two in [128, 8192]");
+    if (had_block == 128 && (K % 128 != 0 || K > 65536))
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "block Hadamard needs K % 128 == 0 and K <= 65536");
+    if (M == 0)
+        return QUAROT_OK;
+    if (!x || !signs || !q || !scales)
+        return fail(QUAROT_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(x) || !aligned16(q) || !aligned16(scales))
+        return fail(QUAROT_ERR_MISALIGNED, "x, q_packed and scales must be 16-byte aligned");
+    return QUAROT_OK;
+}
+
+template <int LOGN, int GROUP>
+quarot_status_t launch_fwht(const void *x, int64_t M, const int8_t *signs, uint8_t *q, void *scales,
+                            cudaStream_t st, int dev, int sms)
+{
+    auto kern = fwht_quant_kernel<LOGN, GROUP>;
+    int per_sm = 0;
+    quarot_status_t s = kernel_occupancy(kern, dev, kFwhtThreads, 0, per_sm);
+    if (s != QUAROT_OK)
+        return s;
+    constexpr int R = kFwhtThreads / ((1 << LOGN) / 128);
+    const int64_t ctas = (M + R - 1) / R;
+    const int grid = (int)std::min<int64_t>(ctas, (int64_t)sms * per_sm);
+    const double n = double(1 << LOGN);
+    kern<<<grid, kFwhtThreads, 0, st>>>(reinterpret_cast<const uint32_t *>(x), M, signs, q, scales,
+                                        (float)(1.0 / (7.0 * std::sqrt(n))), (float)std::sqrt(n));
+    return after_launch("fwht_quant_kernel launch");
+}
+
+template <int GROUP>
+quarot_status_t dispatch_fwht(int logn, const void *x, int64_t M, const int8_t *signs, uint8_t *q,
+                              void *scales, cudaStream_t st, int dev, int sms)
+{
+    switch (logn) {
+    case 8: return launch_fwht<8, GROUP>(x, M, signs, q, scales, st, dev, sms);
+    case 9: return launch_fwht<9, GROUP>(x, M, signs, q, scales, st, dev, sms);
+    case 10: return launch_fwht<10, GROUP>(x, M, signs, q, scales, st, dev, sms);
+    case 11: return launch_fwht<11, GROUP>(x, M, signs, q, scales, st, dev, sms);
+    case 12: return launch_fwht<12, GROUP>(x, M, signs, q, scales, st, dev, sms);
+    case 13: return launch_fwht<13, GROUP>(x, M, signs, q, scales, st, dev, sms);
+    default: return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "unsupported transform size");
+    }
+}
+
+template <bool ROTATE, int GROUP>
+quarot_status_t launch_block(const void *x, int64_t M, int64_t K, const int8_t *signs, uint8_t *q,
+                             void *scales, float scale_mul, float sqrt_n, cudaStream_t st, int dev, int sms)
+{
+    const int nb = (int)(K / 128);
+    const bool multi = nb > kBlockThreads;
+    auto kern = multi ? block128_quant_kernel<ROTATE, GROUP, true> : block128_quant_kernel<ROTATE, GROUP, false>;
+    const int rows_per_cta = multi ? 1 : kBlockThreads / nb;
+    const int threads = multi ? kBlockThreads : ((rows_per_cta * nb + 31) / 32) * 32;
+    int per_sm = 0;
+    quarot_status_t s = kernel_occupancy(kern, dev, threads, 0, per_sm);
+    if (s != QUAROT_OK)
+        return s;
+    const int64_t ctas = (M + rows_per_cta - 1) / rows_per_cta;
+    const int grid = (int)std::min<int64_t>(ctas, (int64_t)sms * per_sm);
+    kern<<<grid, threads, 0, st>>>(reinterpret_cast<const uint4 *>(x), M, (int)K, rows_per_cta, signs, q,
+                                   scales, scale_mul, sqrt_n);
+    return after_launch("block128_quant_kernel launch");
+}
+
+quarot_status_t rotate_quant_launch(const void *x, int64_t M, int64_t K, const int8_t *signs, int had_block,
+                                    int group, uint8_t *q, void *scales, cudaStream_t st)
+{
+    int dev;
+    DeviceInfo *info;
+    quarot_status_t s = current_device(dev, info);
+    if (s != QUAROT_OK)
+        return s;
+    if (had_block == 0 && K >= 256) {
+        const int logn = ilog2(K);
+        return group == 0 ? dispatch_fwht<0>(logn, x, M, signs, q, scales, st, dev, info->sm_count)
+                          : dispatch_fwht<128>(logn, x, M, signs, q, scales, st, dev, info->sm_count);
+    }
+    const float mul = (float)(1.0 / (7.0 * std::sqrt(128.0)));
+    const float sq = (float)std::sqrt(128.0);
+    return group == 0 ? launch_block<true, 0>(x, M, K, signs, q, scales, mul, sq, st, dev, info->sm_count)
+                      : launch_block<true, 128>(x, M, K, signs, q, scales, mul, sq, st, dev, info->sm_count);
+}
+
+// ----------------------------------------------------------------- GEMM
+quarot_status_t check_gemm_args(const void *qa, int64_t M, const void *qw, int64_t N, int64_t K,
+                                const void *out, const void *sa, const void *sw, bool need_scales)
+{
+    if (M < 0 || N <= 0 || K <= 0)
+        return fail(QUAROT_ERR_INVALID_ARG, "M must be >= 0, N and K > 0");
+    if (N % 8 != 0)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "N must be a multiple of 8");
+    if (K % 128 != 0 || K > 65536)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "K must be a multiple of 128 and at most 65536");
+    if (M > (int64_t(1) << 31) - 128 || N > (int64_t(1) << 31) - 256)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "M or N too large");
+    if (M == 0)
+        return QUAROT_OK;
+    if (!qa || !qw || !out || (need_scales && (!sa || !sw)))
+        return fail(QUAROT_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(qa) || !aligned16(qw) || !aligned16(out) || (need_scales && (!aligned16(sa) || !aligned16(sw))))
+        return fail(QUAROT_ERR_MISALIGNED, "operands, scales and output must be 16-byte aligned");
+    return QUAROT_OK;
+}
+
+template <int BN, int EPI>
+quarot_status_t launch_gemm(GemmArgs a, cudaStream_t st, bool pdl)
+{
+    using S = GemmShape<BN, EPI>;
+    int dev;
+    DeviceInfo *info;
+    quarot_status_t s = current_device(dev, info);
+    if (s != QUAROT_OK)
+        return s;
+    auto kern = int4_gemm_kernel<BN, EPI>;
+    int per_sm = 0;
+    s = kernel_occupancy(kern, dev, S::kThreads, S::kSmemBytes, per_sm);
+    if (s != QUAROT_OK)
+        return s;
+    a.tiles_m = (int)((a.M + kGemmBM - 1) / kGemmBM);
+    a.tiles_n = (int)((a.N + BN - 1) / BN);
+    a.kblocks = (int)(a.K / kGemmBK);
+    const int64_t tiles = (int64_t)a.tiles_m * a.tiles_n;
+    if (tiles > 0x7fffffff)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "too many output tiles");
+    const int grid = (int)std::min<int64_t>(tiles, (int64_t)info->sm_count);
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(S::kThreads);
+    cfg.dynamicSmemBytes = S::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    if (pdl) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "int4_gemm_kernel launch");
+    return after_launch("int4_gemm_kernel launch");
+}
+
+quarot_status_t linear_launch(const uint8_t *qa, const void *sa, int64_t M, const uint8_t *qw, const void *sw,
+                              int64_t N, int64_t K, int group, void *out, cudaStream_t st, bool pdl)
+{
+    GemmArgs a = {};
+    a.qa = qa;
+    a.sa = sa;
+    a.qw = qw;
+    a.sw = sw;
+    a.out = out;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    return group == 0 ? launch_gemm<256, kEpiScaledF16>(a, st, pdl) : launch_gemm<128, kEpiGroupF16>(a, st, pdl);
+}
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+}  // namespace
+
+// ======================================================================= C ABI
+extern "C" {
+
+quarot_status_t quarot_rotate_quant(const void *x_f16, int64_t M, int64_t K, const int8_t *signs, int had_block,
+                                    int group, uint8_t *q_packed, void *scales, quarot_stream_t stream)
+{
+    quarot_status_t s = check_rotate_args(x_f16, M, K, signs, had_block, group, q_packed, scales);
+    if (s != QUAROT_OK || M == 0)
+        return s;
+    return rotate_quant_launch(x_f16, M, K, signs, had_block, group, q_packed, scales, (cudaStream_t)stream);
+}
+
+quarot_status_t quarot_int4_linear(const uint8_t *qa, const void *s_a, int64_t M, const uint8_t *qw,
+                                   const void *s_w, int64_t N, int64_t K, int group, void *out_f16,
+                                   quarot_stream_t stream)
+{
+    if (group != 0 && group != 128)
+        return fail(QUAROT_ERR_INVALID_ARG, "group must be 0 or 128");
+    quarot_status_t s = check_gemm_args(qa, M, qw, N, K, out_f16, s_a, s_w, true);
+    if (s != QUAROT_OK || M == 0)
+        return s;
+    return linear_launch(qa, s_a, M, qw, s_w, N, K, group, out_f16, (cudaStream_t)stream, false);
+}
+
+quarot_status_t quarot_int4_gemm_s32(const uint8_t *qa, int64_t M, const uint8_t *qw, int64_t N, int64_t K,
+                                     int32_t *acc, quarot_stream_t stream)
+{
+    quarot_status_t s = check_gemm_args(qa, M, qw, N, K, acc, nullptr, nullptr, false);
+    if (s != QUAROT_OK || M == 0)
+        return s;
+    GemmArgs a = {};
+    a.qa = qa;
+    a.qw = qw;
+    a.out = acc;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    return launch_gemm<256, kEpiS32>(a, (cudaStream_t)stream, false);
+}
+
+size_t quarot_rotate_quant_linear_workspace(int64_t M, int64_t K, int group)
+{
+    if (M <= 0 || K <= 0)
+        return 0;
+    const size_t q = align256((size_t)M * (size_t)(K / 2));
+    const size_t sc = group == 0 ? (size_t)M * 4 : (size_t)M * (size_t)(K / 128) * 2;
+    return q + align256(sc);
+}
+
+quarot_status_t quarot_rotate_quant_linear(const void *x_f16, int64_t M, int64_t K, const int8_t *signs,
+                                           int had_block, int group, const uint8_t *qw, const void *s_w,
+                                           int64_t N, void *workspace, size_t ws_bytes, void *out_f16,
+                                           quarot_stream_t stream)
+{
+    quarot_status_t s = check_rotate_args(x_f16, M, K, signs, had_block, group, workspace, workspace);
+    if (s != QUAROT_OK)
+        return s;
+    s = check_gemm_args(workspace, M, qw, N, K, out_f16, workspace, s_w, true);
+    if (s != QUAROT_OK || M == 0)
+        return s;
+    const size_t need = quarot_rotate_quant_linear_workspace(M, K, group);
+    if (ws_bytes < need)
+        return fail(QUAROT_ERR_INVALID_ARG, "workspace too small");
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(QUAROT_ERR_MISALIGNED, "workspace must be 256-byte aligned");
+    uint8_t *qa = static_cast<uint8_t *>(workspace);
+    void *sa = qa + align256((size_t)M * (size_t)(K / 2));
+    cudaStream_t st = (cudaStream_t)stream;
+    s = rotate_quant_launch(x_f16, M, K, signs, had_block, group, qa, sa, st);
+    if (s != QUAROT_OK)
+        return s;
+    return linear_launch(qa, sa, M, qw, s_w, N, K, group, out_f16, st, true);
+}
+
+quarot_status_t quarot_kv_quant(const void *k_f16, const void *v_f16, int64_t B, int64_t T, int64_t Hkv, int64_t D,
+                                const int8_t *signs, uint8_t *kq, void *ks_f16, uint8_t *vq, void *vs_f16,
+                                quarot_stream_t stream)
+{
+    if (B < 0 || T < 0 || Hkv <= 0)
+        return fail(QUAROT_ERR_INVALID_ARG, "B, T must be >= 0 and Hkv > 0");
+    if (D != 128)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "head dimension must be 128");
+    if (Hkv > 512)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "at most 512 KV heads");
+    const int64_t rows = B * T;
+    if (rows == 0)
+        return QUAROT_OK;
+    if (!k_f16 || !v_f16 || !signs || !kq || !ks_f16 || !vq || !vs_f16)
+        return fail(QUAROT_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(k_f16) || !aligned16(v_f16) || !aligned16(kq) || !aligned16(vq) || !aligned16(ks_f16) ||
+        !aligned16(vs_f16))
+        return fail(QUAROT_ERR_MISALIGNED, "K, V, codes and scales must be 16-byte aligned");
+    int dev;
+    DeviceInfo *info;
+    quarot_status_t s = current_device(dev, info);
+    if (s != QUAROT_OK)
+        return s;
+    const int64_t W = Hkv * D;
+    cudaStream_t st = (cudaStream_t)stream;
+    s = launch_block<true, 128>(k_f16, rows, W, signs, kq, ks_f16, (float)(1.0 / (7.0 * std::sqrt(128.0))),
+                                (float)std::sqrt(128.0), st, dev, info->sm_count);
+    if (s != QUAROT_OK)
+        return s;
+    return launch_block<false, 128>(v_f16, rows, W, nullptr, vq, vs_f16, (float)(1.0 / 7.0), 1.0f, st, dev,
+                                    info->sm_count);
+}
+
+quarot_status_t quarot_kv_decode_scores(const void *q_f16, int64_t B, int64_t Hq, const int8_t *signs,
+                                        const uint8_t *kq, const void *ks_f16, int64_t T, int64_t Hkv, int64_t D,
+                                        float *scores, quarot_stream_t stream)
+{
+    if (B < 0 || T < 0 || Hkv <= 0 || Hq <= 0)
+        return fail(QUAROT_ERR_INVALID_ARG, "B, T must be >= 0; Hq, Hkv > 0");
+    if (D != 128)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "head dimension must be 128");
+    if (Hq % Hkv != 0)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "Hq must be a multiple of Hkv");
+    const int64_t G = Hq / Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "Hq / Hkv must be 1, 2, 4, 8 or 16");
+    if (Hkv > 65535 || B > 65535)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "B and Hkv must be <= 65535");
+    if (B == 0 || T == 0)
+        return QUAROT_OK;
+    if (!q_f16 || !signs || !kq || !ks_f16 || !scores)
+        return fail(QUAROT_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(q_f16) || !aligned16(kq) || !aligned16(ks_f16) || !aligned16(scores))
+        return fail(QUAROT_ERR_MISALIGNED, "q, codes, scales and scores must be 16-byte aligned");
+    int dev;
+    DeviceInfo *info;
+    quarot_status_t s = current_device(dev, info);
+    if (s != QUAROT_OK)
+        return s;
+    const int64_t chunks = (T + kScoreTokPerCta - 1) / kScoreTokPerCta;
+    if (chunks > 0x7fffffff)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "T too large");
+    dim3 grid((unsigned)chunks, (unsigned)Hkv, (unsigned)B);
+    cudaStream_t st = (cudaStream_t)stream;
+    const __half *qh = static_cast<const __half *>(q_f16);
+    const uint4 *k4 = reinterpret_cast<const uint4 *>(kq);
+    const __half *ksh = static_cast<const __half *>(ks_f16);
+    switch (G) {
+    case 1: kv_scores_kernel<1><<<grid, kScoreThreads, 0, st>>>(qh, signs, k4, ksh, T, (int)Hkv, scores); break;
+    case 2: kv_scores_kernel<2><<<grid, kScoreThreads, 0, st>>>(qh, signs, k4, ksh, T, (int)Hkv, scores); break;
+    case 4: kv_scores_kernel<4><<<grid, kScoreThreads, 0, st>>>(qh, signs, k4, ksh, T, (int)Hkv, scores); break;
+    case 8: kv_scores_kernel<8><<<grid, kScoreThreads, 0, st>>>(qh, signs, k4, ksh, T, (int)Hkv, scores); break;
+    default: kv_scores_kernel<16><<<grid, kScoreThreads, 0, st>>>(qh, signs, k4, ksh, T, (int)Hkv, scores); break;
+    }
+    return after_launch("kv_scores_kernel launch");
+}
+
+quarot_status_t quarot_get_device_status(void)
+{
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaDeviceSynchronize");
+    int v = 0;
+    e = cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int));
+    if (e != cudaSuccess)
+        return cuda_fail(e, "read device status");
+    if (v != kDevOk) {
+        const int zero = 0;
+        cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
+        return fail(QUAROT_ERR_DEVICE_TIMEOUT, "a kernel gave up a bounded wait");
+    }
+    return QUAROT_OK;
+}
+
+const char *quarot_status_string(quarot_status_t status)
+{
+    switch (status) {
+    case QUAROT_OK: return "QUAROT_OK";
+    case QUAROT_ERR_INVALID_ARG: return "QUAROT_ERR_INVALID_ARG";
+    case QUAROT_ERR_UNSUPPORTED_SHAPE: return "QUAROT_ERR_UNSUPPORTED_SHAPE";
+    case QUAROT_ERR_MISALIGNED: return "QUAROT_ERR_MISALIGNED";
+    case QUAROT_ERR_CUDA: return "QUAROT_ERR_CUDA";
+    case QUAROT_ERR_DEVICE_TIMEOUT: return "QUAROT_ERR_DEVICE_TIMEOUT";
+    case QUAROT_ERR_NO_DEVICE: return "QUAROT_ERR_NO_DEVICE";
+    }
+    return "QUAROT_ERR_UNKNOWN";
+}
+
+const char *quarot_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

@@ -1,0 +1,333 @@
+// rotate_quant.cuh -- online randomized Hadamard rotation fused with symmetric
+// INT4 round-to-nearest quantization and nibble packing.
+//
+// What it computes (QuaRot summary "Summary" / "Key points": random Hadamard
+// rotations applied online, activations quantized on the fly with RTN,
+// group-wise variant with groups of 128; QuaRot article: randomized Hadamard;
+// DuQuant Knowl 2 / 12: block-diagonal Hadamard of block 128):
+//
+//   x' = (x * diag(s)) * H_n / sqrt(n)   (n = K, or n = 128 block by block)
+//   per-token: scale = max|x'| / 7 (fp32), code = rint(x' / scale)
+//   group-128: scale = fp16(max over the group |x'| / 7),
+//              code = clamp(rint(x' / scale), -8, 7); zero scale -> zero codes
+//   byte i of a row = code[2i] | code[2i+1] << 4
+//
+// Design (HBM-bound: 2 bytes read + 0.5 byte written per element):
+//  * The unnormalized transform y = (x*diag(s)) H_n is computed in fp32
+//    registers; 1/sqrt(n) is folded into the stored scale because the codes
+//    rint(7 y / max|y|) do not depend on it.
+//  * Sign flips are XORs of the fp16 sign bits; each thread packs the signs
+//    of the 128 elements it touches into 4 words once per CTA (the CTAs are
+//    persistent over rows).
+//  * Full transform (n = 2^p, 256 <= n <= 8192): each row is owned by
+//    T = n/128 threads holding 128 values each.  Phase A loads fp16 pairs so
+//    that a thread holds element bit 0 and the top six element bits, and
+//    applies the Walsh-Hadamard along those 7 bits in registers.  A swizzled
+//    shared-memory transpose then gives each thread 128 contiguous elements
+//    (bits 0-6) for phase B, which finishes bits 1..min(6, p-7).  Because
+//    H_n = H_2 (x) ... (x) H_2 (Sylvester), stages along different bits
+//    commute, so the two phases together are exactly H_n.
+//  * Block transform (n = 128): one thread owns one 128-block of a row and
+//    does all 7 stages in registers; no exchange at all.  Rows of more than
+//    128 blocks give each thread several blocks; with a per-token scale the
+//    thread then transforms its blocks twice (once for the row maximum, once
+//    to quantize) instead of keeping them all in registers.
+#pragma once
+
+#include "common.cuh"
+
+namespace quarot {
+
+constexpr int kFwhtThreads = 64;
+constexpr int kBlockThreads = 128;
+
+// Quantizes 128 values of one thread and stores the 64 packed bytes.
+//  GROUP == 0: r = 7 / max|y| of the row; |v r| <= 7 (1 + 2^-23) so the
+//              rounding never leaves [-7, 7] and no clamp is needed.
+//  GROUP != 0: r = 1 / (sqrt(n) * fp16 scale); the clamp matters only when
+//              the fp16 scale is subnormal.
+template <int GROUP>
+__device__ __forceinline__ void quant_pack_store(const float (&v)[128], float r, uint8_t *dst, bool valid)
+{
+    uint32_t pk[16];
+#pragma unroll
+    for (int g = 0; g < 16; ++g) {
+        uint32_t acc = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const float t = v[8 * g + k];
+            uint32_t bits;
+            if (GROUP == 0) {
+                bits = rne_code_bits(t, r);
+            } else {
+                const float z = fminf(fmaxf(t * r, -8.f), 7.f);
+                bits = __float_as_uint(z + 12582912.0f);
+            }
+            acc = push_nibble(acc, bits);
+        }
+        pk[g] = acc;
+    }
+    if (valid) {
+        uint4 *d = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            d[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+    }
+}
+
+// fp16 group scale of a block and the matching code multiplier.
+__device__ __forceinline__ float group_scale(float amax, float scale_mul, float sqrt_n, __half &s16)
+{
+    s16 = __float2half_rn(amax * scale_mul);
+    const float sf = __half2float(s16);
+    return (sf > 0.f && sf <= 65504.f) ? 1.0f / (sf * sqrt_n) : 0.f;
+}
+
+// ---------------------------------------------------------------------------
+// Full transform, K = 2^LOGN with 8 <= LOGN <= 13.
+// ---------------------------------------------------------------------------
+template <int LOGN, int GROUP>
+__global__ void __launch_bounds__(kFwhtThreads, 4)
+fwht_quant_kernel(const uint32_t *__restrict__ x,      // [M, K/2] fp16 pairs
+                  int64_t M, const int8_t *__restrict__ signs,
+                  uint8_t *__restrict__ q,             // [M, K/2]
+                  void *__restrict__ scales,           // fp32 [M] or fp16 [M, K/128]
+                  float scale_mul,                     // 1 / (7 sqrt(K)), rounded to fp32
+                  float sqrt_n)                        // sqrt(K), rounded to fp32
+{
+    static_assert(LOGN >= 8 && LOGN <= 13, "full transform covers 256..8192");
+    constexpr int N = 1 << LOGN;
+    constexpr int T = N / 128;              // threads per row
+    constexpr int R = kFwhtThreads / T;     // rows per CTA iteration
+    constexpr int SH = LOGN - 6;            // element shift of the phase-A pair index j
+    constexpr int PB = (LOGN - 7) < 6 ? (LOGN - 7) : 6;   // phase-B bits 1..PB
+
+    __shared__ __align__(16) float buf[R * N];
+    __shared__ float red[2];
+
+    const int tid = threadIdx.x;
+    const int rl = tid / T;                 // row within the CTA iteration
+    const int tr = tid % T;                 // thread within the row
+    const int key = tid & 31;               // swizzle key of this thread's phase-B row
+
+    // phase A pair j covers elements (j << SH) + 2 tr and the next one
+    uint32_t sgn[4];
+    build_sign_words(signs, [&](int j) { return (j << SH) + 2 * tr; }, sgn);
+
+    for (int64_t row0 = (int64_t)blockIdx.x * R; row0 < M; row0 += (int64_t)gridDim.x * R) {
+        const int64_t row = row0 + rl;
+        const bool valid = row < M;
+        const uint32_t *xr = x + (valid ? row : 0) * (N / 2);
+
+        // ---- phase A: register r = 2 j + b holds element (j << SH) + 2 tr + b
+        float v[128];
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+            const uint32_t w = valid ? __ldg(xr + (j << (SH - 1)) + tr) : 0u;
+            const float2 f = half2_bits_to_float2(apply_sign_pair(w, sgn, j));
+            v[2 * j] = f.x;
+            v[2 * j + 1] = f.y;
+        }
+        fwht_bits<0, 7>(v);
+
+        // ---- transpose through shared memory (16-byte chunks XOR-swizzled)
+        float *rb = buf + rl * N;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+            const int e = (j << SH) + 2 * tr;
+            const int u = e >> 7, c = (e >> 2) & 31, wd = e & 3;
+            const int ukey = (rl * T + u) & 31;
+            *reinterpret_cast<float2 *>(rb + u * 128 + ((c ^ ukey) << 2) + wd) =
+                make_float2(v[2 * j], v[2 * j + 1]);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const float4 f = *reinterpret_cast<const float4 *>(rb + tr * 128 + ((i ^ key) << 2));
+            v[4 * i] = f.x;
+            v[4 * i + 1] = f.y;
+            v[4 * i + 2] = f.z;
+            v[4 * i + 3] = f.w;
+        }
+
+        // ---- phase B: this thread holds elements tr*128 + i, i = 0..127
+        fwht_bits<1, PB + 1>(v);
+
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+            amax = fmaxf(amax, fabsf(v[i]));
+
+        float r;
+        if (GROUP == 0) {
+            if (T <= 32) {
+                amax = warp_max(amax, T);
+                __syncthreads();                      // buffer reads done before reuse
+            } else {
+                amax = warp_max(amax, 32);
+                if ((tid & 31) == 0)
+                    red[tid >> 5] = amax;
+                __syncthreads();
+                amax = fmaxf(red[0], red[1]);
+            }
+            r = amax > 0.f ? 7.0f / amax : 0.f;
+            if (valid && tr == 0)
+                reinterpret_cast<float *>(scales)[row] = amax * scale_mul;
+        } else {
+            __syncthreads();
+            __half s16;
+            r = group_scale(amax, scale_mul, sqrt_n, s16);
+            if (valid)
+                reinterpret_cast<__half *>(scales)[row * (N / 128) + tr] = s16;
+        }
+        quant_pack_store<GROUP>(v, r, q + (valid ? row : 0) * (N / 2) + tr * 64, valid);
+    }
+    // a dependent GEMM launched with programmatic serialization may start now
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Block transform: each thread owns 128-wide blocks of one row.
+//  nb <= 128 blocks per row: one block per thread, 128 / nb rows per CTA.
+//  nb >  128: one row per CTA of 128 threads, blocks b, b+128, ... per thread.
+// ROTATE = false skips the sign flip and the transform (value cache).
+// GROUP = 0: one fp32 scale per row; GROUP = 128: one fp16 scale per block.
+// ---------------------------------------------------------------------------
+template <bool ROTATE>
+__device__ __forceinline__ void load_block(const uint4 *__restrict__ src, bool valid, const uint32_t (&sgn)[4],
+                                           float (&v)[128])
+{
+    uint4 w[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        w[i] = valid ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const uint32_t ww[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint32_t t = ROTATE ? apply_sign_pair(ww[k], sgn, 4 * i + k) : ww[k];
+            const float2 f = half2_bits_to_float2(t);
+            v[8 * i + 2 * k] = f.x;
+            v[8 * i + 2 * k + 1] = f.y;
+        }
+    }
+    if (ROTATE)
+        fwht_bits<0, 7>(v);
+}
+
+template <bool ROTATE, int GROUP, bool MULTI>
+__global__ void __launch_bounds__(kBlockThreads)
+block128_quant_kernel(const uint4 *__restrict__ x,     // [M, K] fp16, 8 per uint4
+                      int64_t M, int K, int rows_per_cta,
+                      const int8_t *__restrict__ signs,
+                      uint8_t *__restrict__ q, void *__restrict__ scales,
+                      float scale_mul, float sqrt_n)
+{
+    constexpr int BPT = MULTI ? 4 : 1;                 // blocks per thread, at most
+    __shared__ unsigned int rowmax[kBlockThreads];
+    __shared__ uint32_t sgn_multi[MULTI ? BPT * 4 * kBlockThreads : 1];   // [block i][word][thread]
+    const int nb = K >> 7;
+    const int tid = threadIdx.x;
+    const int rl = MULTI ? 0 : tid / nb;
+    const int b0 = MULTI ? tid : tid - rl * nb;
+    const bool active = MULTI ? true : rl < rows_per_cta;
+
+    // sign words of this thread's blocks: registers for one block, shared
+    // memory (indexed by block) when a thread owns several
+    uint32_t sgn[4] = {0u, 0u, 0u, 0u};
+    if (!MULTI) {
+        if (ROTATE && active)
+            build_sign_words(signs, [&](int j) { return b0 * 128 + 2 * j; }, sgn);
+    } else {
+#pragma unroll 1
+        for (int i = 0; i < BPT; ++i) {
+            const int b = b0 + i * kBlockThreads;
+            uint32_t t[4] = {0u, 0u, 0u, 0u};
+            if (ROTATE && b < nb)
+                build_sign_words(signs, [&](int j) { return b * 128 + 2 * j; }, t);
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+                sgn_multi[(i * 4 + w) * kBlockThreads + tid] = t[w];
+        }
+    }
+    auto block_signs = [&](int i, uint32_t (&d)[4]) {
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+            d[w] = MULTI ? sgn_multi[(i * 4 + w) * kBlockThreads + tid] : sgn[w];
+    };
+
+    for (int64_t row0 = (int64_t)blockIdx.x * rows_per_cta; row0 < M;
+         row0 += (int64_t)gridDim.x * rows_per_cta) {
+        const int64_t row = row0 + rl;
+        const bool row_ok = active && row < M;
+        const uint4 *xrow = x + (row_ok ? row : 0) * (K / 8);
+        uint8_t *qrow = q + (row_ok ? row : 0) * (K / 2);
+
+        if (GROUP != 0) {
+            // independent blocks
+#pragma unroll 1
+            for (int i = 0; i < BPT; ++i) {
+                const int b = b0 + i * kBlockThreads;
+                const bool ok = row_ok && b < nb;
+                if (MULTI && !__any_sync(0xffffffffu, ok))
+                    break;
+                uint32_t sg[4];
+                block_signs(i, sg);
+                float v[128];
+                load_block<ROTATE>(xrow + (ok ? b : 0) * 16, ok, sg, v);
+                float amax = 0.f;
+#pragma unroll
+                for (int k = 0; k < 128; ++k)
+                    amax = fmaxf(amax, fabsf(v[k]));
+                __half s16;
+                const float r = group_scale(amax, scale_mul, sqrt_n, s16);
+                if (ok)
+                    reinterpret_cast<__half *>(scales)[row * nb + b] = s16;
+                quant_pack_store<GROUP>(v, r, qrow + (ok ? b : 0) * 64, ok);
+            }
+        } else {
+            // one scale per row: reduce the row maximum over the row's threads
+            float v[128];
+            float amax = 0.f;
+#pragma unroll 1
+            for (int i = 0; i < BPT; ++i) {
+                const int b = b0 + i * kBlockThreads;
+                const bool ok = row_ok && b < nb;
+                uint32_t sg[4];
+                block_signs(i, sg);
+                load_block<ROTATE>(xrow + (ok ? b : 0) * 16, ok, sg, v);
+#pragma unroll
+                for (int k = 0; k < 128; ++k)
+                    amax = fmaxf(amax, fabsf(v[k]));
+            }
+            if (tid < rows_per_cta)
+                rowmax[tid] = 0u;
+            __syncthreads();
+            if (active)
+                atomicMax(&rowmax[rl], __float_as_uint(amax));   // amax >= 0: bit order = value order
+            __syncthreads();
+            amax = active ? __uint_as_float(rowmax[rl]) : 0.f;
+            __syncthreads();
+            const float r = amax > 0.f ? 7.0f / amax : 0.f;
+            if (row_ok && b0 == 0)
+                reinterpret_cast<float *>(scales)[row] = amax * scale_mul;
+            if (!MULTI) {
+                quant_pack_store<0>(v, r, qrow + b0 * 64, row_ok);
+            } else {
+#pragma unroll 1
+                for (int i = 0; i < BPT; ++i) {
+                    const int b = b0 + i * kBlockThreads;
+                    const bool ok = row_ok && b < nb;
+                    uint32_t sg[4];
+                    block_signs(i, sg);
+                    load_block<ROTATE>(xrow + (ok ? b : 0) * 16, ok, sg, v);
+                    quant_pack_store<0>(v, r, qrow + (ok ? b : 0) * 64, ok);
+                }
+            }
+        }
+    }
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+}  // namespace quarot

@@ -1,0 +1,89 @@
+"""Parity rules between the CUDA library and the CPU oracle.
+
+ * Integer and byte results (int32 accumulators from identical codes, packed
+   bytes from identical codes) must be bit-exact.
+ * Scales: a per-token / per-channel fp32 scale within 1e-6 relative of the
+   oracle's fp64 max|x'|/7.  An fp16 group scale equal to the oracle's fp16
+   scale, or one fp16 step away only when the oracle's exact max|x'|/7 lies
+   within 1e-5 (relative) of the rounding midpoint between the two: both are
+   then correct roundings of a near-tie.
+ * Codes: once a scale has passed that check, the expected codes are the
+   oracle's RTN of its own fp64 rotated values under that scale.  A device
+   code may differ from them only by +-1, only where the oracle's v/s lies
+   within 1e-3 of a rounding boundary, and in at most 1e-4 of the elements.
+   (The kernel rotates in fp32, the oracle in fp64; the decision can flip
+   only at such near-ties.)
+ * fp16 outputs: max relative error 2e-3 against the oracle's fp64 product,
+   relative to max(|y_ref|, 1e-2 * rms(y_ref row)) so that outputs near zero
+   (which any rounding order perturbs by more than 2e-3 of themselves) are
+   judged on the row's scale.
+"""
+import numpy as np
+
+import oracle
+
+
+def unpack_codes(packed) -> np.ndarray:
+    return oracle.unpack(np.asarray(packed, np.uint8))
+
+
+def check_scales(gpu_scales, xr, group):
+    """Returns the device scales as fp64 once they pass the scale rule."""
+    M, K = xr.shape
+    if group == 0:
+        amax = np.abs(xr).max(axis=1)
+        ref = amax / 7.0
+        got = np.asarray(gpu_scales, np.float64)
+        rel = np.abs(got - ref) / np.maximum(ref, 1e-300)
+        bad = (rel > 1e-6) & ~((ref == 0) & (got == 0))
+        assert not np.any(bad), f"per-token scales off: max rel {rel[bad].max():.3e} at rows {np.nonzero(bad)[0][:5]}"
+        return got
+    G = K // group
+    amax = np.abs(xr.reshape(M, G, group)).max(axis=2)
+    exact = amax / 7.0
+    ref16 = oracle.f64_to_f16(exact)
+    got16 = np.asarray(gpu_scales).view(np.uint16).reshape(M, G)
+    diff = got16.astype(np.int64) - ref16.astype(np.int64)
+    off = diff != 0
+    if np.any(off):
+        assert np.all(np.abs(diff[off]) == 1), "fp16 scales more than one step off"
+        a = oracle.f16_to_f64(got16[off])
+        b = oracle.f16_to_f64(ref16[off])
+        mid = (a + b) / 2
+        near = np.abs(exact[off] - mid) <= 1e-5 * np.abs(mid)
+        assert np.all(near), "fp16 scale differs from the oracle away from a rounding near-tie"
+    return got16
+
+
+def check_codes(gpu_packed, gpu_scales, xr, group, max_frac=1e-4):
+    """Applies the scale and code rules; returns the number of near-tie flips."""
+    sc = check_scales(gpu_scales, xr, group)
+    expect = oracle.quantize_with_scales(xr, sc, group)
+    got = unpack_codes(gpu_packed).reshape(xr.shape)
+    d = got.astype(np.int16) - expect.astype(np.int16)
+    flips = d != 0
+    n = int(flips.sum())
+    if n == 0:
+        return 0
+    assert np.all(np.abs(d[flips]) == 1), "codes differ by more than one step"
+    M, K = xr.shape
+    s = oracle.scales_to_f64(sc)
+    s_el = np.repeat(s.reshape(M, -1), K if group == 0 else group, axis=1)
+    t = np.where(s_el > 0, xr / np.where(s_el > 0, s_el, 1.0), 0.0)
+    dist = np.abs(t - (np.floor(t) + 0.5))
+    assert np.all(dist[flips] < 1e-3), f"code flips away from near-ties (max dist {dist[flips].max():.3e})"
+    assert n <= max_frac * got.size, f"{n} code flips in {got.size} elements"
+    return n
+
+
+def check_f16_output(y_gpu_f16, y_ref, tol=2e-3):
+    y = np.asarray(y_gpu_f16, np.float16).astype(np.float64)
+    ref = np.asarray(y_ref, np.float64)
+    rms = np.sqrt(np.mean(ref * ref, axis=-1, keepdims=True))
+    denom = np.maximum(np.abs(ref), 1e-2 * rms)
+    denom = np.where(denom > 0, denom, 1.0)
+    err = np.abs(y - ref) / denom
+    assert np.all(np.isfinite(y)), "non-finite outputs"
+    worst = float(err.max()) if err.size else 0.0
+    assert worst <= tol, f"max relative error {worst:.3e} > {tol}"
+    return worst

@@ -417,3 +417,17 @@ def test_kv_scores_spike_query_closed_form():
         expect = c * s[h, j] * Hm[j].sum() / np.sqrt(D) * 7 * 0.25
         assert abs(got[0, hq, 1] - expect) <= 1e-12
         assert got[0, hq, 0] == 0 and got[0, hq, 2] == 0
+
+
+def test_quantize_with_given_scales_matches_own_scales():
+    # with the oracle's own scales the two routes agree; with halved scales codes saturate
+    x = synth.random_f16((4, 256), 50)
+    xr = oracle.rotate(x, synth.signs(256, 50), 0)
+    codes, sc = oracle.quantize(xr, 0)
+    np.testing.assert_array_equal(oracle.quantize_with_scales(xr, sc, 0), codes)
+    xg = oracle.rotate(x, synth.signs(256, 51), 128)
+    cg, sg = oracle.quantize(xg, 128)
+    np.testing.assert_array_equal(oracle.quantize_with_scales(xg, sg, 128), cg)
+    half = oracle.quantize_with_scales(xr, sc / 2, 0)
+    j = np.argmax(np.abs(xr), axis=1)
+    assert set(np.unique(half[np.arange(4), j])) <= {-8, 7}
