@@ -12,7 +12,11 @@
    code may differ from them only by +-1, only where the oracle's v/s lies
    within 1e-3 of a rounding boundary, and in at most 1e-4 of the elements.
    (The kernel rotates in fp32, the oracle in fp64; the decision can flip
-   only at such near-ties.)
+   only at such near-ties.)  Values lying exactly on a boundary (v/s = k + 1/2
+   to fp64 precision, which structured inputs such as constant rows produce
+   in bulk) have two correct roundings -- any perturbation of s in either
+   direction picks one -- so either is accepted there and such elements are
+   not counted against the 1e-4 budget.
  * fp16 outputs: max relative error 2e-3 against the oracle's fp64 product,
    relative to max(|y_ref|, 1e-2 * rms(y_ref row)) so that outputs near zero
    (which any rounding order perturbs by more than 2e-3 of themselves) are
@@ -72,7 +76,16 @@ def check_codes(gpu_packed, gpu_scales, xr, group, max_frac=1e-4):
     t = np.where(s_el > 0, xr / np.where(s_el > 0, s_el, 1.0), 0.0)
     dist = np.abs(t - (np.floor(t) + 0.5))
     assert np.all(dist[flips] < 1e-3), f"code flips away from near-ties (max dist {dist[flips].max():.3e})"
-    assert n <= max_frac * got.size, f"{n} code flips in {got.size} elements"
+    # exact ties are judged with the oracle's own scale (fp64 max|x'|/7 per row,
+    # or the checked fp16 group scale)
+    if group == 0:
+        s0 = np.abs(xr).max(axis=1, keepdims=True) / 7.0
+        t0 = np.where(s0 > 0, xr / np.where(s0 > 0, s0, 1.0), 0.0)
+    else:
+        t0 = t
+    exact_tie = np.abs(t0 - (np.floor(t0) + 0.5)) <= 1e-9 * np.maximum(1.0, np.abs(t0))
+    counted = int((flips & ~exact_tie).sum())
+    assert counted <= max_frac * got.size, f"{counted} near-tie code flips in {got.size} elements"
     return n
 
 
