@@ -145,6 +145,46 @@ quarot_status_t quarot_rotate_quant_linear(const void *x_f16, int64_t M, int64_t
                                            quarot_stream_t stream);
 
 /*
+ * quarot_rotate_quant_linear_noalloc -- quarot_rotate_quant_linear for callers
+ * that cannot give this library any device memory.  No passage of the pages
+ * corresponds to this entry point; it exists for how the library is called,
+ * not for the method.
+ *
+ * Who needs it: code that reaches the kernels only through this C interface
+ * and has no device allocator of its own to draw a workspace from (a host
+ * program or plug-in whose device memory belongs to another framework), and
+ * serving loops whose device memory was budgeted up front and that must not
+ * call cudaMalloc / cudaFree on the request path -- those calls can
+ * synchronize the device and can fail under memory pressure in the middle of
+ * a request.  This call allocates nothing: no cudaMalloc, no cudaFree, no
+ * allocating library routine.
+ *
+ * Instead of a caller workspace it uses a scratch array compiled into the
+ * library: QUAROT_NOALLOC_SCRATCH_BYTES (16 MiB) of device memory that every
+ * GPU which loads the library holds until the process exits.  Sizes whose
+ * workspace, quarot_rotate_quant_linear_workspace(M, K, group), is larger
+ * return QUAROT_ERR_UNSUPPORTED_SHAPE (with per-token scales, 16 MiB holds
+ * up to 4092 tokens at K = 8192, or 8176 tokens at K = 4096).
+ *
+ * The first call on a device looks up the array's device address with that
+ * device current (cudaGetSymbolAddress) and keeps it; make that first call
+ * before any stream capture.  All calls share the one array, which keeps the
+ * last call's contents; nothing in it has to start at zero, because the
+ * quantizer writes every byte the GEMM then reads.  Calls that can overlap on
+ * the GPU (other streams, or unordered host threads) race on the array: the
+ * caller must serialize them.
+ *
+ * Arguments, layouts, limits and results are those of
+ * quarot_rotate_quant_linear without `workspace` and `ws_bytes`; the output is
+ * the same.
+ */
+#define QUAROT_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+quarot_status_t quarot_rotate_quant_linear_noalloc(const void *x_f16, int64_t M, int64_t K,
+                                                   const int8_t *signs, int had_block, int group,
+                                                   const uint8_t *qw, const void *s_w, int64_t N,
+                                                   void *out_f16, quarot_stream_t stream);
+
+/*
  * quarot_kv_quant -- INT4 KV-cache write [QR-A: the KV cache in 4 bits;
  * DQ-12: fixed Hadamard on the query-key product, per-head quantization].
  *

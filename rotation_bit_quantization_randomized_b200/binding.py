@@ -34,6 +34,7 @@ _SIGS = {
     "quarot_int4_gemm_s32": ([_P, _I64, _P, _I64, _I64, _P, _P], _INT),
     "quarot_rotate_quant_linear_workspace": ([_I64, _I64, _INT], _SZ),
     "quarot_rotate_quant_linear": ([_P, _I64, _I64, _P, _INT, _INT, _P, _P, _I64, _P, _SZ, _P, _P], _INT),
+    "quarot_rotate_quant_linear_noalloc": ([_P, _I64, _I64, _P, _INT, _INT, _P, _P, _I64, _P, _P], _INT),
     "quarot_kv_quant": ([_P, _P, _I64, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P], _INT),
     "quarot_kv_decode_scores": ([_P, _I64, _I64, _P, _P, _P, _I64, _I64, _I64, _P, _P], _INT),
     "quarot_get_device_status": ([], _INT),
@@ -153,6 +154,19 @@ def quarot_rotate_quant_linear(x: torch.Tensor, signs: torch.Tensor, qw: torch.T
            lib.quarot_rotate_quant_linear(_ptr(x), M, K, _ptr(signs), had_block, group, _ptr(qw), _ptr(s_w), N,
                                           _ptr(workspace), workspace.numel() * workspace.element_size(),
                                           _ptr(out), _stream(stream)))
+    return out
+
+
+def quarot_rotate_quant_linear_noalloc(x: torch.Tensor, signs: torch.Tensor, qw: torch.Tensor,
+                                       s_w: torch.Tensor, out: torch.Tensor, had_block: int = 0, group: int = 0,
+                                       stream=None):
+    """The fused path on the library's built-in scratch; the caller supplies every
+    buffer, including `out` (fp16 [M, N]), and nothing is allocated."""
+    M, K = x.shape
+    N = qw.shape[0]
+    _check("quarot_rotate_quant_linear_noalloc",
+           lib.quarot_rotate_quant_linear_noalloc(_ptr(x), M, K, _ptr(signs), had_block, group, _ptr(qw),
+                                                  _ptr(s_w), N, _ptr(out), _stream(stream)))
     return out
 
 

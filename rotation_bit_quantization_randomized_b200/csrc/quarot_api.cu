@@ -291,6 +291,28 @@ quarot_status_t linear_launch(const uint8_t *qa, const void *sa, int64_t M, cons
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
+// Scratch of quarot_rotate_quant_linear_noalloc: a fixed device array that
+// every GPU loading the library holds until exit.  In host code the name is
+// only a host-side handle, never a device address: the kernels get the
+// address cudaGetSymbolAddress returns, looked up once per device.
+constexpr size_t kNoAllocScratchBytes = size_t(QUAROT_NOALLOC_SCRATCH_BYTES);
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+void *g_noalloc_addr[kMaxDevices];
+
+quarot_status_t noalloc_scratch_address(int dev, void *&addr)
+{
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if (!g_noalloc_addr[dev]) {
+        void *p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cudaGetSymbolAddress of the built-in scratch");
+        g_noalloc_addr[dev] = p;
+    }
+    addr = g_noalloc_addr[dev];
+    return QUAROT_OK;
+}
+
 }  // namespace
 
 // ======================================================================= C ABI
@@ -359,6 +381,40 @@ quarot_status_t quarot_rotate_quant_linear(const void *x_f16, int64_t M, int64_t
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return fail(QUAROT_ERR_MISALIGNED, "workspace must be 256-byte aligned");
     uint8_t *qa = static_cast<uint8_t *>(workspace);
+    void *sa = qa + align256((size_t)M * (size_t)(K / 2));
+    cudaStream_t st = (cudaStream_t)stream;
+    s = rotate_quant_launch(x_f16, M, K, signs, had_block, group, qa, sa, st);
+    if (s != QUAROT_OK)
+        return s;
+    return linear_launch(qa, sa, M, qw, s_w, N, K, group, out_f16, st, true);
+}
+
+quarot_status_t quarot_rotate_quant_linear_noalloc(const void *x_f16, int64_t M, int64_t K, const int8_t *signs,
+                                                   int had_block, int group, const uint8_t *qw, const void *s_w,
+                                                   int64_t N, void *out_f16, quarot_stream_t stream)
+{
+    // the scratch stands in for the quantized activations and their scales
+    quarot_status_t s = check_rotate_args(x_f16, M, K, signs, had_block, group, out_f16, out_f16);
+    if (s != QUAROT_OK)
+        return s;
+    s = check_gemm_args(out_f16, M, qw, N, K, out_f16, out_f16, s_w, true);
+    if (s != QUAROT_OK || M == 0)
+        return s;
+    const size_t need = quarot_rotate_quant_linear_workspace(M, K, group);
+    if (need > kNoAllocScratchBytes)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE,
+                    "these sizes need " + std::to_string(need) + " bytes of scratch; the built-in scratch holds " +
+                        std::to_string(kNoAllocScratchBytes) + " (QUAROT_NOALLOC_SCRATCH_BYTES)");
+    int dev;
+    DeviceInfo *info;
+    s = current_device(dev, info);
+    if (s != QUAROT_OK)
+        return s;
+    void *scratch = nullptr;
+    s = noalloc_scratch_address(dev, scratch);
+    if (s != QUAROT_OK)
+        return s;
+    uint8_t *qa = static_cast<uint8_t *>(scratch);
     void *sa = qa + align256((size_t)M * (size_t)(K / 2));
     cudaStream_t st = (cudaStream_t)stream;
     s = rotate_quant_launch(x_f16, M, K, signs, had_block, group, qa, sa, st);
