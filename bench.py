@@ -45,7 +45,9 @@ def parse():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--e2e-steps", type=int, default=3)
-    p.add_argument("--cpu-rows", type=int, default=192, help="token rows of the CPU-baseline sample")
+    p.add_argument("--cpu-rows", type=int, default=2048, help="token rows of the CPU-baseline sample")
+    p.add_argument("--case", choices=["gemm", "gemm_group", "rotate", "block", "kvquant", "kvscores"],
+                   default=None, help="time one kernel on a capture-sized workload (for ncu), not the step")
     return p.parse_args()
 
 
@@ -381,8 +383,74 @@ def run_ours(args, rank, world, local_rank, dist):
         print(json.dumps(line))
 
 
+def run_case(args):
+    """One kernel on a smaller, capture-sized case; random codes/values drawn on the device."""
+    import torch
+    from rotation_bit_quantization_randomized_b200 import binding as q
+    torch.manual_seed(0)
+    dev = torch.device("cuda:0")
+    g = torch.Generator(device=dev)
+    g.manual_seed(1234)
+    if args.case in ("gemm", "gemm_group"):
+        M, N, K = 4096, 28672, 8192
+        group = 128 if args.case == "gemm_group" else 0
+        qa = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=dev, generator=g)
+        qw = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=dev, generator=g)
+        if group:
+            sa = (torch.rand((M, K // 128), device=dev, generator=g) + 0.5).half()
+            sw = (torch.rand((N, K // 128), device=dev, generator=g) * 1e-3 + 1e-3).half()
+        else:
+            sa = torch.rand((M,), device=dev, generator=g) + 0.5
+            sw = torch.rand((N,), device=dev, generator=g) * 1e-3 + 1e-3
+        out = torch.empty((M, N), dtype=torch.float16, device=dev)
+        fn = lambda: q.quarot_int4_linear(qa, sa, qw, sw, group, out)
+        work, unit = 2.0 * M * N * K / 1e12, "TOPS"
+    elif args.case in ("rotate", "block"):
+        M, K = (8192, 8192) if args.case == "rotate" else (8192, 11008)
+        hb, group = (0, 0) if args.case == "rotate" else (128, 128)
+        x = torch.randn((M, K), device=dev, generator=g).half()
+        s = (torch.randint(0, 2, (K,), device=dev, generator=g) * 2 - 1).to(torch.int8)
+        qa = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+        sa = torch.empty((M,), dtype=torch.float32, device=dev) if group == 0 else \
+            torch.empty((M, K // 128), dtype=torch.float16, device=dev)
+        fn = lambda: q.quarot_rotate_quant(x, s, hb, group, qa, sa)
+        work, unit = bytes_rotate_quant(M, K) / 1e9, "GB/s"
+    else:
+        B, T, H, D, Hq = 16, 2048, 8, 128, 64
+        k = torch.randn((B, T, H, D), device=dev, generator=g).half()
+        v = torch.randn((B, T, H, D), device=dev, generator=g).half()
+        qh = torch.randn((B, Hq, D), device=dev, generator=g).half()
+        s = (torch.randint(0, 2, (H, D), device=dev, generator=g) * 2 - 1).to(torch.int8)
+        kq, ks, vq, vs = q.quarot_kv_quant(k, v, s)
+        scores = torch.empty((B, Hq, T), dtype=torch.float32, device=dev)
+        if args.case == "kvquant":
+            fn = lambda: q.quarot_kv_quant(k, v, s, kq, ks, vq, vs)
+            work = bytes_kv_quant(B, T, H, D) / 1e9
+        else:
+            fn = lambda: q.quarot_kv_decode_scores(qh, s, kq, ks, scores)
+            work = bytes_kv_scores(B, T, H, D, Hq) / 1e9
+        unit = "GB/s"
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    if q.quarot_get_device_status() != 0:
+        raise RuntimeError("device status not OK")
+    ms = e0.elapsed_time(e1) / args.steps
+    print(json.dumps({"case": args.case, "ms": ms, unit: work / (ms * 1e-3), "source_sha": source_hash()}))
+
+
 def main():
     args = parse()
+    if args.case:
+        run_case(args)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -11,26 +11,35 @@
 //   out[m, n]  = fp16(sum_g acc_g[m, n] * s_a[m, g] * s_w[n, g])   (groups of 128)
 //
 // Kernel structure (persistent, one CTA per SM, warp-specialized):
-//  * loader warps (each thread owns two tile rows of A or B): read 64 packed
-//    bytes of each row per 128-wide K block straight from global memory
-//    (prefetched two blocks ahead into registers), widen each nibble to
-//    an int8 equal to 16 * code (the nibble lands in the top half of its
-//    byte, so the sign comes for free), and store them into a 4-stage ring in
-//    the 128-byte-swizzled K-major layout the tensor core reads.  Inside each
+//  * TMA producer (one thread): per 128-wide K block, two tiled bulk-tensor
+//    copies bring the packed A tile (128 rows x 64 B) and B tile (BN rows x
+//    64 B) into a ring of packed stages; rows past M or N arrive as zeros.
+//    The copy engine keeps many blocks in flight without the per-SM limits
+//    of ordinary loads.
+//  * unpack warps: read a packed stage (16 B per lane, 8 rows x 64 B per warp
+//    instruction), widen each nibble to an int8 equal to 16 * code (the
+//    nibble lands in the top half of its byte, so the sign comes for free),
+//    store the ring of int8 stages, and only then release the packed stage
+//    to the copy engine (its reads are complete once their values have been
+//    stored).  The int8 stages use the 128-byte-swizzled K-major layout the
+//    tensor core reads.  Inside each
 //    32-wide K chunk the widened order is [low nibbles, high nibbles]; A and B
 //    use the same order, so every dot product is unchanged.  Both operands
 //    are scaled by 16, so the accumulator holds 256 * acc, removed exactly in
 //    the epilogue (|256 acc| <= 2^14 K < 2^31 for K <= 65536).
-//  * one MMA thread: waits for a full stage, issues four 128 x BN x 32
-//    tcgen05.mma, and commits to the stage's "empty" barrier; at the end of a
+//  * one MMA thread: waits for a full int8 stage, issues four 128 x BN x 32
+//    tcgen05.mma and commits to the stage's "empty" barrier; at the end of a
 //    tile it commits to the accumulator's "full" barrier.  Two accumulator
 //    buffers in tensor memory let the epilogue of tile i overlap the
 //    mainloop of tile i+1.
 //  * epilogue warps: tcgen05.ld the accumulator (warp w reads TMEM lanes
 //    32(w%4)..+31 = tile rows), scale, convert, store.
 //  * every wait is bounded in time; on expiry the CTA records a timeout in
-//    the device status word, drains its issued MMAs and frees tensor memory.
+//    the device status word, drains its issued copies and MMAs and frees
+//    tensor memory.
 #pragma once
+
+#include <cuda.h>
 
 #include "common.cuh"
 #include "tc_ptx.cuh"
@@ -41,31 +50,41 @@ enum : int { kEpiScaledF16 = 0, kEpiS32 = 1, kEpiGroupF16 = 2 };
 
 constexpr int kGemmBM = 128;
 constexpr int kGemmBK = 128;            // int8 elements of K per stage (one 128-byte row)
-constexpr int kGemmStages = 4;
-constexpr int kGemmPrefetch = 2;        // K blocks a loader has in flight ahead of its stores
 constexpr int kGemmGroupM = 16;         // tiles along M that share a band of N tiles
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 template <int BN, int EPI>
 struct GemmShape {
-    static constexpr int kABytes = kGemmBM * kGemmBK;
+    static constexpr int kPackedA = kGemmBM * kGemmBK / 2;       // bytes of a packed A block
+    static constexpr int kPackedB = BN * kGemmBK / 2;
+    static constexpr int kPackedStage = kPackedA + kPackedB;
+    static constexpr int kABytes = kGemmBM * kGemmBK;            // widened int8 A block
     static constexpr int kBBytes = BN * kGemmBK;
     static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kLoadRows = kGemmBM + BN;      // A rows then B rows of a tile
-    static constexpr int kLoadThreads = kLoadRows / 2;  // two rows per loader thread
+    static constexpr int kPStages = BN == 256 ? 3 : 4;           // packed ring
+    static constexpr int kIStages = BN == 256 ? 3 : 4;           // int8 ring
+    static constexpr int kLoadRows = kGemmBM + BN;               // A rows then B rows of a tile
+    static constexpr int kGroupsPerWarp = 8;                     // 8 rows per warp instruction
+    static constexpr int kUnpackWarps = kLoadRows / (8 * kGroupsPerWarp);
+    static constexpr int kUnpackThreads = 32 * kUnpackWarps;
     static constexpr int kEpiWarps = EPI == kEpiGroupF16 ? 8 : 4;
     static constexpr int kEpiThreads = 32 * kEpiWarps;
     static constexpr int kMmaWarp = kEpiWarps;
-    static constexpr int kLoadWarp0 = kEpiWarps + 1;
-    static constexpr int kThreads = 32 * (kEpiWarps + 1) + kLoadThreads;
+    static constexpr int kTmaWarp = kEpiWarps + 1;
+    static constexpr int kUnpackWarp0 = kEpiWarps + 2;
+    static constexpr int kThreads = 32 * (kUnpackWarp0 + kUnpackWarps);
     static constexpr int kTmemCols = 2 * BN;
-    static constexpr int kBarOffset = kGemmStages * kStageBytes;
-    static constexpr int kNumBars = 2 * kGemmStages + 7;
+    static constexpr int kIntOffset = kPStages * kPackedStage;  // int8 ring after the packed ring
+    static constexpr int kBarOffset = kIntOffset + kIStages * kStageBytes;
+    static constexpr int kNumBars = 2 * kPStages + 2 * kIStages + 7;
     static constexpr int kMiscOffset = kBarOffset + 8 * kNumBars;
     static constexpr int kSwOffset = kMiscOffset + 16;
     static constexpr int kSmemBytes = kSwOffset + 2 * BN * 4 + 1024;
-    static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
+    static_assert(kStageBytes % 1024 == 0 && kIntOffset % 1024 == 0, "int8 stages keep 1024-byte alignment");
+    static_assert(kPackedStage % 1024 == 0, "packed stages keep 1024-byte alignment");
+    static_assert(kGemmBM % (8 * kGroupsPerWarp) == 0, "an unpack warp handles only A or only B rows");
     static_assert(kTmemCols == 256 || kTmemCols == 512, "TMEM allocation is a power of two");
+    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
 struct GemmArgs {
@@ -112,7 +131,7 @@ __device__ __forceinline__ bool gemm_wait(uint32_t bar, uint32_t parity, volatil
     }
 }
 
-// Bounded wait that ignores the abort flag (used to drain issued MMAs).
+// Bounded wait that ignores the abort flag (used to drain issued work).
 __device__ __forceinline__ bool gemm_wait_drain(uint32_t bar, uint32_t parity)
 {
     const uint64_t t0 = globaltimer_ns();
@@ -135,15 +154,18 @@ __device__ __forceinline__ float small_i2f(uint32_t v)
 
 template <int BN, int EPI>
 __global__ void __launch_bounds__(GemmShape<BN, EPI>::kThreads, 1)
-int4_gemm_kernel(const GemmArgs a)
+int4_gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_a,
+                 const __grid_constant__ CUtensorMap tma_b)
 {
     using S = GemmShape<BN, EPI>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t bar_full = sbase + S::kBarOffset;
-    const uint32_t bar_empty = bar_full + 8 * kGemmStages;
-    const uint32_t bar_accf = bar_empty + 8 * kGemmStages;
+    const uint32_t bar_pfull = sbase + S::kBarOffset;
+    const uint32_t bar_pempty = bar_pfull + 8 * S::kPStages;
+    const uint32_t bar_ifull = bar_pempty + 8 * S::kPStages;
+    const uint32_t bar_iempty = bar_ifull + 8 * S::kIStages;
+    const uint32_t bar_accf = bar_iempty + 8 * S::kIStages;
     const uint32_t bar_acce = bar_accf + 16;
     const uint32_t bar_drain = bar_acce + 16;
     const uint32_t bar_sws = bar_drain + 8;        // grouped: column-scale staging, 2 buffers
@@ -155,11 +177,16 @@ int4_gemm_kernel(const GemmArgs a)
     const int num_tiles = a.tiles_m * a.tiles_n;
     const int KB = a.kblocks;
     const int my_tiles = blockIdx.x < num_tiles ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const int total = my_tiles * KB;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kGemmStages; ++s) {
-            mbar_init(bar_full + 8 * s, S::kLoadThreads);
-            mbar_init(bar_empty + 8 * s, 1);
+        for (int s = 0; s < S::kPStages; ++s) {
+            mbar_init(bar_pfull + 8 * s, 1);
+            mbar_init(bar_pempty + 8 * s, S::kUnpackThreads);
+        }
+        for (int s = 0; s < S::kIStages; ++s) {
+            mbar_init(bar_ifull + 8 * s, S::kUnpackThreads);
+            mbar_init(bar_iempty + 8 * s, 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar_accf + 8 * b, 1);
@@ -184,81 +211,87 @@ int4_gemm_kernel(const GemmArgs a)
     // dependent launch); everything above overlapped its tail
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    if (warp >= S::kLoadWarp0) {
-        // ------------------------------------------------------------ loaders
-        // thread l owns rows l and l + kLoadThreads of the combined
-        // [A rows 0..127 | B rows 0..BN-1] index space
-        const int l = threadIdx.x - 32 * S::kLoadWarp0;
-        const int64_t ldb = a.K / 2;
-        const int total = my_tiles * KB;
-        int rrow[2];
-        bool isA[2];
-        uint32_t row_off[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int c = l + h * S::kLoadThreads;
-            isA[h] = c < kGemmBM;
-            rrow[h] = isA[h] ? c : c - kGemmBM;
-            row_off[h] = (isA[h] ? 0u : (uint32_t)S::kABytes) + (rrow[h] >> 3) * 1024 + (rrow[h] & 7) * 128;
-        }
-
-        auto fetch = [&](uint4 (&d)[2][4], int step) {
-            const int lt = step / KB;
-            const int kb = step - lt * KB;
-            int mb, nb;
-            gemm_tile_coords(blockIdx.x + lt * gridDim.x, a.tiles_m, a.tiles_n, mb, nb);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int64_t row = (int64_t)(isA[h] ? mb * kGemmBM : nb * BN) + rrow[h];
-                const bool ok = row < (isA[h] ? a.M : a.N);
-                const uint4 *p = reinterpret_cast<const uint4 *>((isA[h] ? a.qa : a.qw) + (ok ? row : 0) * ldb +
-                                                                 (int64_t)kb * 64);
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    d[h][c] = ok ? __ldg(p + c) : make_uint4(0, 0, 0, 0);
-            }
-        };
-
-        uint4 pf[kGemmPrefetch][2][4];
-#pragma unroll
-        for (int p = 0; p < kGemmPrefetch; ++p)
-            if (p < total)
-                fetch(pf[p], p);
-
-        bool ok = true;
-        static_assert(kGemmStages % kGemmPrefetch == 0, "unrolled ring indexing");
-        for (int it = 0; it < total && ok; it += kGemmStages) {
-#pragma unroll
-            for (int p = 0; p < kGemmStages; ++p) {
-                const int step = it + p;          // stage index == p
-                const int slot = p % kGemmPrefetch;
-                if (step < total && ok) {
-                    const uint32_t use = (uint32_t)(step / kGemmStages);
-                    if (!gemm_wait(bar_empty + 8 * p, (use & 1) ^ 1, abort_flag)) {
-                        ok = false;
-                    } else {
-#pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            uint8_t *dst = smem + p * S::kStageBytes + row_off[h];
-                            const int sw = rrow[h] & 7;
-#pragma unroll
-                            for (int c = 0; c < 4; ++c) {
-                                const uint4 w = pf[slot][h][c];
-                                const uint4 lo = make_uint4((w.x << 4) & 0xF0F0F0F0u, (w.y << 4) & 0xF0F0F0F0u,
-                                                            (w.z << 4) & 0xF0F0F0F0u, (w.w << 4) & 0xF0F0F0F0u);
-                                const uint4 hi = make_uint4(w.x & 0xF0F0F0F0u, w.y & 0xF0F0F0F0u,
-                                                            w.z & 0xF0F0F0F0u, w.w & 0xF0F0F0F0u);
-                                *reinterpret_cast<uint4 *>(dst + (((2 * c) ^ sw) << 4)) = lo;
-                                *reinterpret_cast<uint4 *>(dst + (((2 * c + 1) ^ sw) << 4)) = hi;
-                            }
-                        }
-                        fence_proxy_async_smem();
-                        mbar_arrive(bar_full + 8 * p);
-                        if (step + kGemmPrefetch < total)
-                            fetch(pf[slot], step + kGemmPrefetch);
-                    }
+    if (warp == S::kTmaWarp) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tma_a);
+            tma_prefetch_desc(&tma_b);
+            int lt = 0, kb = 0, mb = 0, nb = 0;
+            if (total > 0)
+                gemm_tile_coords(blockIdx.x, a.tiles_m, a.tiles_n, mb, nb);
+            int step = 0;
+            for (; step < total; ++step) {
+                const int ps = step % S::kPStages;
+                const uint32_t use = (uint32_t)(step / S::kPStages);
+                if (!gemm_wait(bar_pempty + 8 * ps, (use & 1) ^ 1, abort_flag))
+                    break;
+                const uint32_t dst = sbase + ps * S::kPackedStage;
+                mbar_arrive_expect_tx(bar_pfull + 8 * ps, S::kPackedStage);
+                tma_load_2d(dst, &tma_a, kb * (kGemmBK / 2), mb * kGemmBM, bar_pfull + 8 * ps);
+                tma_load_2d(dst + S::kPackedA, &tma_b, kb * (kGemmBK / 2), nb * BN, bar_pfull + 8 * ps);
+                if (++kb == KB) {
+                    kb = 0;
+                    if (++lt < my_tiles)
+                        gemm_tile_coords(blockIdx.x + lt * gridDim.x, a.tiles_m, a.tiles_n, mb, nb);
                 }
             }
+            // copies into stages the unpackers never consumed (abort only) land
+            // before the CTA exits
+            for (int s = step - S::kPStages; s < step; ++s)
+                if (s >= 0)
+                    gemm_wait_drain(bar_pfull + 8 * (s % S::kPStages), (uint32_t)(s / S::kPStages) & 1);
+        }
+        __syncwarp();
+    } else if (warp >= S::kUnpackWarp0) {
+        // ------------------------------------------------------------ unpackers
+        // Unpack warp uw owns row groups 8 uw .. 8 uw + 7 of the combined
+        // [A rows 0..127 | B rows 0..BN-1] index space; in each group lane
+        // (r, c) = (lane / 4, lane % 4) handles 16 packed bytes (32 codes) of
+        // row 8 g + r, which become the row's 16-byte int8 chunks 2c (low
+        // nibbles) and 2c + 1 (high nibbles).
+        const int uw = warp - S::kUnpackWarp0;
+        const int rsub = lane >> 2;
+        const int csub = lane & 3;
+        const int row0 = 8 * S::kGroupsPerWarp * uw;
+        const bool isA = row0 < kGemmBM;                          // warp-uniform
+        const int tile_row0 = isA ? row0 : row0 - kGemmBM;        // row inside the A or B tile
+        const uint32_t p_off = isA ? 0u : (uint32_t)S::kPackedA;
+        const uint32_t i_off = isA ? 0u : (uint32_t)S::kABytes;
+        for (int step = 0; step < total; ++step) {
+            const int ps = step % S::kPStages;
+            const int is = step % S::kIStages;
+            if (!gemm_wait(bar_pfull + 8 * ps, (uint32_t)(step / S::kPStages) & 1, abort_flag))
+                break;
+            uint4 w[S::kGroupsPerWarp];
+            const uint8_t *src = smem + ps * S::kPackedStage + p_off;
+#pragma unroll
+            for (int j = 0; j < S::kGroupsPerWarp; ++j) {
+                const int r = tile_row0 + 8 * j + rsub;
+                w[j] = *reinterpret_cast<const uint4 *>(src + r * (kGemmBK / 2) + csub * 16);
+            }
+            if (!gemm_wait(bar_iempty + 8 * is, ((uint32_t)(step / S::kIStages) & 1) ^ 1, abort_flag))
+                break;
+            uint8_t *st_base = smem + S::kIntOffset + is * S::kStageBytes + i_off;
+#pragma unroll
+            for (int j = 0; j < S::kGroupsPerWarp; ++j) {
+                const int r = tile_row0 + 8 * j + rsub;
+                uint8_t *dst = st_base + (r >> 3) * 1024 + (r & 7) * 128;
+                const int sw = r & 7;
+                const uint4 v = w[j];
+                const uint4 lo = make_uint4((v.x << 4) & 0xF0F0F0F0u, (v.y << 4) & 0xF0F0F0F0u,
+                                            (v.z << 4) & 0xF0F0F0F0u, (v.w << 4) & 0xF0F0F0F0u);
+                const uint4 hi = make_uint4(v.x & 0xF0F0F0F0u, v.y & 0xF0F0F0F0u,
+                                            v.z & 0xF0F0F0F0u, v.w & 0xF0F0F0F0u);
+                *reinterpret_cast<uint4 *>(dst + (((2 * csub) ^ sw) << 4)) = lo;
+                *reinterpret_cast<uint4 *>(dst + (((2 * csub + 1) ^ sw) << 4)) = hi;
+            }
+            // The packed stage is released only now: its values have been
+            // consumed by the stores above, so the shared-memory reads are
+            // complete, and the proxy fence orders them before the copy
+            // engine's next write into the stage.
+            fence_proxy_async_smem();
+            mbar_arrive(bar_ifull + 8 * is);
+            mbar_arrive(bar_pempty + 8 * ps);
         }
     } else if (warp == S::kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
@@ -277,14 +310,13 @@ int4_gemm_kernel(const GemmArgs a)
                         }
                         tc_fence_after();
                     }
-                    const int stage = step % kGemmStages;
-                    const uint32_t use = (uint32_t)(step / kGemmStages);
-                    if (!gemm_wait(bar_full + 8 * stage, use & 1, abort_flag)) {
+                    const int is = step % S::kIStages;
+                    if (!gemm_wait(bar_ifull + 8 * is, (uint32_t)(step / S::kIStages) & 1, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t as = sbase + stage * S::kStageBytes;
+                    const uint32_t as = sbase + S::kIntOffset + is * S::kStageBytes;
                     const uint32_t bs = as + S::kABytes;
                     const uint32_t d = tmem_base + ab * BN;
 #pragma unroll
@@ -292,7 +324,7 @@ int4_gemm_kernel(const GemmArgs a)
                         const uint32_t acc = (EPI == kEpiGroupF16) ? (j > 0) : (kb > 0 || j > 0);
                         umma_i8_ss(d, desc_kmajor_sw128(as + 32 * j), desc_kmajor_sw128(bs + 32 * j), idesc, acc);
                     }
-                    umma_commit(bar_empty + 8 * stage);
+                    umma_commit(bar_iempty + 8 * is);
                     if (EPI == kEpiGroupF16 || kb == KB - 1)
                         umma_commit(bar_accf + 8 * ab);
                 }

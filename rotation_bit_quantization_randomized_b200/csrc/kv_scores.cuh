@@ -57,53 +57,63 @@ kv_scores_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
     __syncthreads();
 
     const int64_t t0 = (int64_t)blockIdx.x * kScoreTokPerCta + tid;
-    uint32_t code[kScoreTokPerThread][16];
+    const uint4 *src[kScoreTokPerThread];
+    bool tok_ok[kScoreTokPerThread];
     float acc[kScoreTokPerThread][G];
 #pragma unroll
     for (int i = 0; i < kScoreTokPerThread; ++i) {
         const int64_t t = t0 + (int64_t)i * kScoreThreads;
-        const bool ok = t < T;
-        const uint4 *src = kq + ((b * T + (ok ? t : 0)) * Hkv + h) * 4;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            uint4 w = ok ? __ldg(src + c) : make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
-            code[i][4 * c] = w.x;
-            code[i][4 * c + 1] = w.y;
-            code[i][4 * c + 2] = w.z;
-            code[i][4 * c + 3] = w.w;
-        }
+        tok_ok[i] = t < T;
+        src[i] = kq + ((b * T + (tok_ok[i] ? t : 0)) * Hkv + h) * 4;
 #pragma unroll
         for (int g = 0; g < G; ++g)
             acc[i][g] = 0.f;
     }
 
+    // 16 bytes (32 codes) of every token per iteration; the loop is not
+    // unrolled so that the body stays in the instruction cache
+    uint4 cur[kScoreTokPerThread];
 #pragma unroll
-    for (int wd = 0; wd < 16; ++wd) {
+    for (int i = 0; i < kScoreTokPerThread; ++i)
+        cur[i] = tok_ok[i] ? __ldg(src[i]) : make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
+#pragma unroll 1
+    for (int qd = 0; qd < 4; ++qd) {
+        uint4 nx[kScoreTokPerThread];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const int d = wd * 8 + k;
-            float qv[G];
+        for (int i = 0; i < kScoreTokPerThread; ++i)
+            nx[i] = (qd < 3 && tok_ok[i]) ? __ldg(src[i] + qd + 1) : cur[i];
 #pragma unroll
-            for (int g = 0; g < G; g += 4) {
-                if (G >= 4) {
-                    float4 f = *reinterpret_cast<const float4 *>(&qs[d][g]);
-                    qv[g] = f.x; qv[g + 1] = f.y; qv[g + 2] = f.z; qv[g + 3] = f.w;
-                } else {
+        for (int wd = 0; wd < 4; ++wd) {
 #pragma unroll
-                    for (int gg = 0; gg < G; ++gg)
-                        qv[gg] = qs[d][gg];
+            for (int k = 0; k < 8; ++k) {
+                const int d = qd * 32 + wd * 8 + k;
+                float qv[G];
+#pragma unroll
+                for (int g = 0; g < G; g += 4) {
+                    if (G >= 4) {
+                        const float4 f = *reinterpret_cast<const float4 *>(&qs[d][g]);
+                        qv[g] = f.x; qv[g + 1] = f.y; qv[g + 2] = f.z; qv[g + 3] = f.w;
+                    } else {
+#pragma unroll
+                        for (int gg = 0; gg < G; ++gg)
+                            qv[gg] = qs[d][gg];
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < kScoreTokPerThread; ++i) {
+                    const uint32_t word = wd == 0 ? cur[i].x : wd == 1 ? cur[i].y : wd == 2 ? cur[i].z : cur[i].w;
+                    // nibble -> float exactly: (2^23 + (c ^ 8)) - (2^23 + 8) = c
+                    const uint32_t u = ((word >> (4 * k)) & 0xFu) ^ 0x4B000008u;
+                    const float c = __uint_as_float(u) - 8388616.0f;
+#pragma unroll
+                    for (int g = 0; g < G; ++g)
+                        acc[i][g] = fmaf(qv[g], c, acc[i][g]);
                 }
             }
-#pragma unroll
-            for (int i = 0; i < kScoreTokPerThread; ++i) {
-                // nibble -> float exactly: (2^23 + (c ^ 8)) - (2^23 + 8) = c
-                const uint32_t u = ((code[i][wd] >> (4 * k)) & 0xFu) ^ 0x4B000008u;
-                const float c = __uint_as_float(u) - 8388616.0f;
-#pragma unroll
-                for (int g = 0; g < G; ++g)
-                    acc[i][g] = fmaf(qv[g], c, acc[i][g]);
-            }
         }
+#pragma unroll
+        for (int i = 0; i < kScoreTokPerThread; ++i)
+            cur[i] = nx[i];
     }
 
 #pragma unroll

@@ -8,6 +8,8 @@
 #include "kv_scores.cuh"
 #include "rotate_quant.cuh"
 
+#include <cuda.h>
+
 #include <cmath>
 #include <cstdio>
 #include <mutex>
@@ -234,6 +236,50 @@ quarot_status_t check_gemm_args(const void *qa, int64_t M, const void *qw, int64
     return QUAROT_OK;
 }
 
+// cuTensorMapEncodeTiled, fetched from the driver through the runtime so that
+// the library does not link libcuda directly.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+quarot_status_t encode_tiled_fn(EncodeTiledFn &fn)
+{
+    static EncodeTiledFn cached = nullptr;
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if (!cached) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)");
+        if (q != cudaDriverEntryPointSuccess || !p)
+            return fail(QUAROT_ERR_CUDA, "the driver does not provide cuTensorMapEncodeTiled");
+        cached = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    fn = cached;
+    return QUAROT_OK;
+}
+
+// Tensor map of a packed INT4 matrix [rows, K/2] bytes read in boxes of
+// 64 bytes (128 codes) x box_rows rows; rows past the end read as zeros.
+quarot_status_t packed_map(CUtensorMap &map, const uint8_t *base, int64_t rows, int64_t K, int box_rows)
+{
+    EncodeTiledFn fn;
+    quarot_status_t s = encode_tiled_fn(fn);
+    if (s != QUAROT_OK)
+        return s;
+    const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+    const cuuint32_t box[2] = {(cuuint32_t)(kGemmBK / 2), (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(QUAROT_ERR_CUDA, "cuTensorMapEncodeTiled failed (code " + std::to_string((int)r) + ")");
+    return QUAROT_OK;
+}
+
 template <int BN, int EPI>
 quarot_status_t launch_gemm(GemmArgs a, cudaStream_t st, bool pdl)
 {
@@ -254,6 +300,13 @@ quarot_status_t launch_gemm(GemmArgs a, cudaStream_t st, bool pdl)
     const int64_t tiles = (int64_t)a.tiles_m * a.tiles_n;
     if (tiles > 0x7fffffff)
         return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "too many output tiles");
+    CUtensorMap map_a, map_b;
+    s = packed_map(map_a, a.qa, a.M, a.K, kGemmBM);
+    if (s != QUAROT_OK)
+        return s;
+    s = packed_map(map_b, a.qw, a.N, a.K, BN);
+    if (s != QUAROT_OK)
+        return s;
     const int grid = (int)std::min<int64_t>(tiles, (int64_t)info->sm_count);
 
     cudaLaunchConfig_t cfg = {};
@@ -268,7 +321,7 @@ quarot_status_t launch_gemm(GemmArgs a, cudaStream_t st, bool pdl)
         cfg.attrs = attr;
         cfg.numAttrs = 1;
     }
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a, map_a, map_b);
     if (e != cudaSuccess)
         return cuda_fail(e, "int4_gemm_kernel launch");
     return after_launch("int4_gemm_kernel launch");

@@ -114,20 +114,34 @@ fwht_quant_kernel(const uint32_t *__restrict__ x,      // [M, K/2] fp16 pairs
     uint32_t sgn[4];
     build_sign_words(signs, [&](int j) { return (j << SH) + 2 * tr; }, sgn);
 
-    for (int64_t row0 = (int64_t)blockIdx.x * R; row0 < M; row0 += (int64_t)gridDim.x * R) {
+    // raw fp16 pairs of the next row this thread handles: loaded one row ahead
+    // so that the loads overlap the transform of the current row
+    uint32_t nxt[64];
+    auto load_row = [&](int64_t r0) {
+        const int64_t r = r0 + rl;
+        const bool ok = r < M;
+        const uint32_t *xr = x + (ok ? r : 0) * (N / 2);
+#pragma unroll
+        for (int j = 0; j < 64; ++j)
+            nxt[j] = ok ? __ldg(xr + (j << (SH - 1)) + tr) : 0u;
+    };
+    const int64_t stride = (int64_t)gridDim.x * R;
+    load_row((int64_t)blockIdx.x * R);
+
+    for (int64_t row0 = (int64_t)blockIdx.x * R; row0 < M; row0 += stride) {
         const int64_t row = row0 + rl;
         const bool valid = row < M;
-        const uint32_t *xr = x + (valid ? row : 0) * (N / 2);
 
         // ---- phase A: register r = 2 j + b holds element (j << SH) + 2 tr + b
         float v[128];
 #pragma unroll
         for (int j = 0; j < 64; ++j) {
-            const uint32_t w = valid ? __ldg(xr + (j << (SH - 1)) + tr) : 0u;
-            const float2 f = half2_bits_to_float2(apply_sign_pair(w, sgn, j));
+            const float2 f = half2_bits_to_float2(apply_sign_pair(nxt[j], sgn, j));
             v[2 * j] = f.x;
             v[2 * j + 1] = f.y;
         }
+        if (row0 + stride < M)
+            load_row(row0 + stride);
         fwht_bits<0, 7>(v);
 
         // ---- transpose through shared memory (16-byte chunks XOR-swizzled)
