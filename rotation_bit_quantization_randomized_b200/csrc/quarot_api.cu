@@ -5,6 +5,7 @@
 
 #include "common.cuh"
 #include "int4_gemm.cuh"
+#include "int4_gemm_pair.cuh"
 #include "kv_scores.cuh"
 #include "rotate_quant.cuh"
 
@@ -327,6 +328,60 @@ quarot_status_t launch_gemm(GemmArgs a, cudaStream_t st, bool pdl)
     return after_launch("int4_gemm_kernel launch");
 }
 
+// The per-token / per-channel GEMM on CTA pairs (clusters of two).
+template <int EPI>
+quarot_status_t launch_gemm_pair(GemmArgs a, cudaStream_t st, bool pdl)
+{
+    using S = PairShape<EPI>;
+    int dev;
+    DeviceInfo *info;
+    quarot_status_t s = current_device(dev, info);
+    if (s != QUAROT_OK)
+        return s;
+    auto kern = int4_gemm_pair_kernel<EPI>;
+    int per_sm = 0;
+    s = kernel_occupancy(kern, dev, S::kThreads, S::kSmemBytes, per_sm);
+    if (s != QUAROT_OK)
+        return s;
+    a.tiles_m = (int)((a.M + kPairBM - 1) / kPairBM);
+    a.tiles_n = (int)((a.N + kPairBN - 1) / kPairBN);
+    a.kblocks = (int)(a.K / kGemmBK);
+    const int64_t tiles = (int64_t)a.tiles_m * a.tiles_n;
+    if (tiles > 0x7fffffff)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "too many output tiles");
+    CUtensorMap map_a, map_b;
+    s = packed_map(map_a, a.qa, a.M, a.K, S::kRows);
+    if (s != QUAROT_OK)
+        return s;
+    s = packed_map(map_b, a.qw, a.N, a.K, S::kRows);
+    if (s != QUAROT_OK)
+        return s;
+    const int clusters = (int)std::min<int64_t>(tiles, (int64_t)(info->sm_count / 2));
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * clusters);
+    cfg.blockDim = dim3(S::kThreads);
+    cfg.dynamicSmemBytes = S::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    int nattr = 1;
+    if (pdl) {
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        nattr = 2;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = nattr;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a, map_a, map_b);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "int4_gemm_pair_kernel launch");
+    return after_launch("int4_gemm_pair_kernel launch");
+}
+
 quarot_status_t linear_launch(const uint8_t *qa, const void *sa, int64_t M, const uint8_t *qw, const void *sw,
                               int64_t N, int64_t K, int group, void *out, cudaStream_t st, bool pdl)
 {
@@ -339,7 +394,7 @@ quarot_status_t linear_launch(const uint8_t *qa, const void *sa, int64_t M, cons
     a.M = M;
     a.N = N;
     a.K = K;
-    return group == 0 ? launch_gemm<256, kEpiScaledF16>(a, st, pdl) : launch_gemm<128, kEpiGroupF16>(a, st, pdl);
+    return group == 0 ? launch_gemm_pair<kEpiScaledF16>(a, st, pdl) : launch_gemm<128, kEpiGroupF16>(a, st, pdl);
 }
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -405,7 +460,7 @@ quarot_status_t quarot_int4_gemm_s32(const uint8_t *qa, int64_t M, const uint8_t
     a.M = M;
     a.N = N;
     a.K = K;
-    return launch_gemm<256, kEpiS32>(a, (cudaStream_t)stream, false);
+    return launch_gemm_pair<kEpiS32>(a, (cudaStream_t)stream, false);
 }
 
 size_t quarot_rotate_quant_linear_workspace(int64_t M, int64_t K, int group)
