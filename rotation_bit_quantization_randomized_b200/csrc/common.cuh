@@ -118,6 +118,23 @@ __device__ __forceinline__ float2 half2_bits_to_float2(uint32_t bits)
     return __half22float2(h);
 }
 
+// max(a, b, c): the three-input form of sm_100 (one instruction).
+__device__ __forceinline__ float max3f(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// (d0, d1) = (a0 * b + c, a1 * b + c) with one packed fp32x2 fused multiply-add.
+__device__ __forceinline__ void fma_x2(float a0, float a1, float b, float c, float &d0, float &d1)
+{
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\t"
+        "mov.b64 rc, {%5, %5};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+
 __device__ __forceinline__ float warp_max(float v, int width)
 {
 #pragma unroll

@@ -53,17 +53,21 @@ __device__ __forceinline__ void quant_pack_store(const float (&v)[128], float r,
 #pragma unroll
     for (int g = 0; g < 16; ++g) {
         uint32_t acc = 0;
+        if (GROUP == 0) {
+            // two codes per packed fma: rint(t r) lands in the low mantissa bits
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const float t = v[8 * g + k];
-            uint32_t bits;
-            if (GROUP == 0) {
-                bits = rne_code_bits(t, r);
-            } else {
-                const float z = fminf(fmaxf(t * r, -8.f), 7.f);
-                bits = __float_as_uint(z + 12582912.0f);
+            for (int k = 0; k < 8; k += 2) {
+                float f0, f1;
+                fma_x2(v[8 * g + k], v[8 * g + k + 1], r, 12582912.0f, f0, f1);
+                acc = push_nibble(acc, __float_as_uint(f0));
+                acc = push_nibble(acc, __float_as_uint(f1));
             }
-            acc = push_nibble(acc, bits);
+        } else {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const float z = fminf(fmaxf(v[8 * g + k] * r, -8.f), 7.f);
+                acc = push_nibble(acc, __float_as_uint(z + 12582912.0f));
+            }
         }
         pk[g] = acc;
     }
@@ -169,8 +173,8 @@ fwht_quant_kernel(const uint32_t *__restrict__ x,      // [M, K/2] fp16 pairs
 
         float amax = 0.f;
 #pragma unroll
-        for (int i = 0; i < 128; ++i)
-            amax = fmaxf(amax, fabsf(v[i]));
+        for (int i = 0; i < 128; i += 2)
+            amax = max3f(amax, fabsf(v[i]), fabsf(v[i + 1]));
 
         float r;
         if (GROUP == 0) {
@@ -292,8 +296,8 @@ block128_quant_kernel(const uint4 *__restrict__ x,     // [M, K] fp16, 8 per uin
                 load_block<ROTATE>(xrow + (ok ? b : 0) * 16, ok, sg, v);
                 float amax = 0.f;
 #pragma unroll
-                for (int k = 0; k < 128; ++k)
-                    amax = fmaxf(amax, fabsf(v[k]));
+                for (int k = 0; k < 128; k += 2)
+                    amax = max3f(amax, fabsf(v[k]), fabsf(v[k + 1]));
                 __half s16;
                 const float r = group_scale(amax, scale_mul, sqrt_n, s16);
                 if (ok)
@@ -312,8 +316,8 @@ block128_quant_kernel(const uint4 *__restrict__ x,     // [M, K] fp16, 8 per uin
                 block_signs(i, sg);
                 load_block<ROTATE>(xrow + (ok ? b : 0) * 16, ok, sg, v);
 #pragma unroll
-                for (int k = 0; k < 128; ++k)
-                    amax = fmaxf(amax, fabsf(v[k]));
+                for (int k = 0; k < 128; k += 2)
+                    amax = max3f(amax, fabsf(v[k]), fabsf(v[k + 1]));
             }
             if (tid < rows_per_cta)
                 rowmax[tid] = 0u;
