@@ -300,7 +300,7 @@ def run_ours(args, rank, world, local_rank, dist):
     rq_gbs = bytes_rotate_quant(M, K) / (k_ms[0] * 1e-3) / 1e9
     kvq_gbs = bytes_kv_quant(c.B, c.T, c.Hkv, c.D) / (k_ms[2] * 1e-3) / 1e9
     kvs_gbs = bytes_kv_scores(c.B, c.T, c.Hkv, c.D, c.Hq) / (k_ms[3] * 1e-3) / 1e9
-    traffic = recorded_traffic("int4_gemm_kernel")
+    traffic = recorded_traffic("int4_gemm_pair_kernel")
 
     # ---- end to end through the public API with host buffers (rank-local)
     x_p = torch.from_numpy(x_h).pin_memory()
@@ -361,7 +361,7 @@ def run_ours(args, rank, world, local_rank, dist):
             "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N, "kv": [c.B, c.T, c.Hkv, c.D], "q_heads": c.Hq,
                        "l2": "inputs and outputs larger than L2; no explicit flush",
                        "parallelism": f"replicas x{world}"},
-            "roofline": {"bound": "tensor", "kernel": "int4_gemm_kernel (quarot_int4_linear)",
+            "roofline": {"bound": "tensor", "kernel": "int4_gemm_pair_kernel<0> (quarot_int4_linear)",
                          "achieved": gemm_tops, "peak": int8_sust, "unit": "TFLOP/s",
                          "frac": gemm_tops / int8_sust, "traffic": traffic,
                          "peak_note": f"int8 dense = 2 x bf16 sustained {pk['bf16_sust']} {pk['src']}"},
