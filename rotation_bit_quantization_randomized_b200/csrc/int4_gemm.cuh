@@ -131,6 +131,14 @@ __device__ __forceinline__ bool gemm_wait(uint32_t bar, uint32_t parity, volatil
     }
 }
 
+// Warp-uniform bounded wait: the warp goes on only if every lane saw the
+// phase complete, so after a timeout no lane reaches a warp-collective
+// tcgen05 instruction without the others.
+__device__ __forceinline__ bool gemm_wait_warp(uint32_t bar, uint32_t parity, volatile int *abort_flag)
+{
+    return __all_sync(0xffffffffu, gemm_wait(bar, parity, abort_flag));
+}
+
 // Bounded wait that ignores the abort flag (used to drain issued work).
 __device__ __forceinline__ bool gemm_wait_drain(uint32_t bar, uint32_t parity)
 {

@@ -1,25 +1,48 @@
 // int4_gemm_pair.cuh -- the per-token / per-channel INT4 linear layer on CTA
-// pairs: tcgen05.mma.cta_group::2 computes 256 x 256 output tiles, each CTA of
-// the pair holding 128 rows of A and 128 rows (its half of the N tile) of B.
+// pairs: tcgen05.mma.cta_group::2 computes 256 x BN output tiles; each CTA of
+// the pair holds 128 rows of A and BN/2 rows (its half of the N tile) of B.
 //
-// Same method and data flow as int4_gemm.cuh (TMA of packed tiles, nibble
-// widening by unpack warps, int8 tensor-core MMA into tensor memory, fused
-// dequantizing epilogue); what changes is that each SM now stages and widens
-// half of the B tile instead of all of it, which cuts the shared-memory
-// traffic per multiply-add by a third -- the kernel's bound.
+// Same method as int4_gemm.cuh (TMA of packed tiles, nibble widening, int8
+// tensor-core MMA with int32 accumulation in tensor memory, fused
+// dequantizing epilogue).  The kernel is bound by shared-memory bandwidth, so
+// the operands take different routes:
+//  * A (activations): each unpack thread owns one A row; it reads the row's
+//    64 packed bytes (the TMA writes them with the 64-byte swizzle, so the
+//    per-row reads of a warp hit distinct banks), widens them in registers
+//    and writes the 128 int8 values straight into tensor memory with
+//    tcgen05.st (lane = row).  The MMA reads A from tensor memory: A never
+//    passes through shared memory in widened form.
+//  * B (weights): widened into the 128-byte-swizzled K-major shared-memory
+//    stage the MMA reads, as in the single-CTA kernel, but only the CTA's
+//    half of the N tile.
+//
+// Tensor memory (512 columns per CTA): two accumulator buffers of BN columns
+// at 0 and BN, then the int8 A stages of 32 columns (128 K values) each; the
+// number of stages is what the remaining columns hold.
+//
+// Stages: a ring of 8 packed stages (TMA -> unpackers), 4 int8 B stages in
+// shared memory and kAStages = (512 - 2 BN) / 32 int8 A stages in tensor
+// memory.  Two groups of four unpack warps take alternate K steps.  A group
+// reads and widens step s, stores its B half as soon as the MMAs of step
+// s - 4 are done, and only then waits for the MMAs of step s - kAStages to
+// free its A stage: after that wait comes nothing but the tensor-memory store
+// and the arrival, so the stage hand-off the tensor core waits on is short.
 //
 // Pair protocol (CTA rank 0 = leader):
 //  * each CTA's TMA producer fills its own packed ring; its unpack warps fill
-//    its own int8 ring and, after a proxy fence, every unpack thread of both
-//    CTAs arrives on the LEADER's "int8 stage full" barrier;
+//    its own A stage (tensor memory) and B stage (shared memory) and, after
+//    the store waits, fences and a warp barrier, lane 0 of every unpack warp
+//    of both CTAs arrives on the LEADER's "int8 stage full" barrier;
 //  * the leader's MMA thread issues the pair MMAs and commits with a
-//    multicast to the "stage empty" / "accumulator full" barriers of both
-//    CTAs;
+//    multicast to the "step done" / "accumulator full" barriers of both
+//    CTAs (MMAs complete in order, so "step s done" also frees the stages of
+//    every earlier step);
 //  * each CTA's epilogue reads its own 128 accumulator rows and arrives on
 //    the leader's "accumulator empty" barrier;
 //  * a cluster barrier precedes the release of tensor memory, so neither CTA
-//    leaves while its peer may still read its shared memory or signal it.
-// All waits are bounded in time, as in the single-CTA kernel.
+//    leaves while its peer may still read its memory or signal it.
+// All waits are bounded in time, as in the single-CTA kernel; waits in front
+// of warp-collective tcgen05 instructions are warp-uniform.
 #pragma once
 
 #include "int4_gemm.cuh"
@@ -27,49 +50,58 @@
 namespace quarot {
 
 constexpr int kPairBM = 256;       // output rows per CTA pair
-constexpr int kPairBN = 256;       // output columns per CTA pair
 
-template <int EPI>
+template <int BN, int EPI>
 struct PairShape {
-    static constexpr int kRows = 128;                                 // A rows and B rows per CTA
-    static constexpr int kPackedA = kRows * kGemmBK / 2;
-    static constexpr int kPackedStage = 2 * kPackedA;
-    static constexpr int kABytes = kRows * kGemmBK;
-    static constexpr int kStageBytes = 2 * kABytes;
-    static constexpr int kPStages = 4;
-    static constexpr int kIStages = 4;
-    static constexpr int kGroupsPerWarp = 8;
-    static constexpr int kUnpackWarps = 2 * kRows / (8 * kGroupsPerWarp);   // 4
-    static constexpr int kUnpackThreads = 32 * kUnpackWarps;
+    static constexpr int kRowsA = kPairBM / 2;                        // A rows per CTA
+    static constexpr int kRowsB = BN / 2;                             // B rows per CTA
+    static constexpr int kPackedA = kRowsA * kGemmBK / 2;             // 8 KB, 64-byte swizzled
+    static constexpr int kPackedB = kRowsB * kGemmBK / 2;
+    static constexpr int kPackedStage = kPackedA + kPackedB;
+    static constexpr int kBBytes = kRowsB * kGemmBK;                  // widened B stage
+    static constexpr int kTmemCols = 512;
+    static constexpr int kAStages = (kTmemCols - 2 * BN) / 32;       // int8 A stages in tensor memory
+    static constexpr int kBStages = 4;                                // int8 B stages in shared memory
+    static constexpr int kPStages = 8;
+    static constexpr int kBGroups = kRowsB / 8;                       // groups of 8 B rows
+    static constexpr int kUnpackWarps = 4;                            // per group: one per TMEM lane quarter
+    static constexpr int kUnpackGroups = 2;                           // groups take alternate K steps
+    static constexpr int kBGroupsPerWarp = (kBGroups + kUnpackWarps - 1) / kUnpackWarps;
+    static constexpr int kUnpackArrivals = kUnpackWarps;              // one arrival per warp and stage
     static constexpr int kEpiWarps = 4;
     static constexpr int kMmaWarp = 4;
     static constexpr int kTmaWarp = 5;
     static constexpr int kUnpackWarp0 = 6;
-    static constexpr int kThreads = 32 * (kUnpackWarp0 + kUnpackWarps);
-    static constexpr int kTmemCols = 2 * kPairBN;                     // two accumulator buffers
+    static constexpr int kThreads = 32 * (kUnpackWarp0 + kUnpackGroups * kUnpackWarps);
+    static constexpr int kACol0 = 2 * BN;                             // A stage s at kACol0 + 32 s
     static constexpr int kIntOffset = kPStages * kPackedStage;
-    static constexpr int kBarOffset = kIntOffset + kIStages * kStageBytes;
-    static constexpr int kNumBars = 2 * kPStages + 2 * kIStages + 5;
+    static constexpr int kBarOffset = kIntOffset + kBStages * kBBytes;
+    static constexpr int kNumBars = 2 * kPStages + 2 * kBStages + 5;
     static constexpr int kMiscOffset = kBarOffset + 8 * kNumBars;
     static constexpr int kSmemBytes = kMiscOffset + 16 + 1024;
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
-    static_assert(kStageBytes % 1024 == 0 && kIntOffset % 1024 == 0, "1024-byte aligned int8 stages");
+    static_assert(kPackedStage % 1024 == 0 && kBBytes % 1024 == 0, "1024-byte aligned stages");
+    static_assert(kRowsB % 8 == 0 && BN % 32 == 0 && BN <= 256, "B rows in groups of 8; N tile of whole column chunks");
+    static_assert(kAStages >= kUnpackGroups && kACol0 + 32 * kAStages <= kTmemCols, "tensor-memory plan");
+    static_assert(kBStages >= kAStages && kBStages % kAStages == 0, "an A stage is free once its B stage is");
+    static_assert(kPStages % kUnpackGroups == 0 && kBStages % kUnpackGroups == 0,
+                  "each stage barrier is used by one unpack group");
 };
 
-template <int EPI>
-__global__ void __launch_bounds__(PairShape<EPI>::kThreads, 1)
+template <int BN, int EPI>
+__global__ void __launch_bounds__(PairShape<BN, EPI>::kThreads, 1)
 int4_gemm_pair_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_a,
                       const __grid_constant__ CUtensorMap tma_b)
 {
-    using S = PairShape<EPI>;
+    using S = PairShape<BN, EPI>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
     const uint32_t bar_pfull = sbase + S::kBarOffset;
     const uint32_t bar_pempty = bar_pfull + 8 * S::kPStages;
     const uint32_t bar_ifull = bar_pempty + 8 * S::kPStages;       // used in the leader
-    const uint32_t bar_iempty = bar_ifull + 8 * S::kIStages;
-    const uint32_t bar_accf = bar_iempty + 8 * S::kIStages;
+    const uint32_t bar_sdone = bar_ifull + 8 * S::kBStages;        // MMAs of step s done (slot s % kBStages)
+    const uint32_t bar_accf = bar_sdone + 8 * S::kBStages;
     const uint32_t bar_acce = bar_accf + 16;                       // used in the leader
     const uint32_t bar_drain = bar_acce + 16;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + S::kMiscOffset);
@@ -89,11 +121,11 @@ int4_gemm_pair_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_
     if (threadIdx.x == 0) {
         for (int s = 0; s < S::kPStages; ++s) {
             mbar_init(bar_pfull + 8 * s, 1);
-            mbar_init(bar_pempty + 8 * s, S::kUnpackThreads);
+            mbar_init(bar_pempty + 8 * s, S::kUnpackArrivals);
         }
-        for (int s = 0; s < S::kIStages; ++s) {
-            mbar_init(bar_ifull + 8 * s, 2 * S::kUnpackThreads);    // leader's: both CTAs' unpackers
-            mbar_init(bar_iempty + 8 * s, 1);
+        for (int s = 0; s < S::kBStages; ++s) {
+            mbar_init(bar_ifull + 8 * s, 2 * S::kUnpackArrivals);   // leader's: both CTAs' unpackers
+            mbar_init(bar_sdone + 8 * s, 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar_accf + 8 * b, 1);
@@ -131,8 +163,8 @@ int4_gemm_pair_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_
                     break;
                 const uint32_t dst = sbase + ps * S::kPackedStage;
                 mbar_arrive_expect_tx(bar_pfull + 8 * ps, S::kPackedStage);
-                tma_load_2d(dst, &tma_a, kb * (kGemmBK / 2), mb * kPairBM + S::kRows * rank, bar_pfull + 8 * ps);
-                tma_load_2d(dst + S::kPackedA, &tma_b, kb * (kGemmBK / 2), nb * kPairBN + S::kRows * rank,
+                tma_load_2d(dst, &tma_a, kb * (kGemmBK / 2), mb * kPairBM + S::kRowsA * rank, bar_pfull + 8 * ps);
+                tma_load_2d(dst + S::kPackedA, &tma_b, kb * (kGemmBK / 2), nb * BN + S::kRowsB * rank,
                             bar_pfull + 8 * ps);
                 if (++kb == KB) {
                     kb = 0;
@@ -147,54 +179,98 @@ int4_gemm_pair_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_
         __syncwarp();
     } else if (warp >= S::kUnpackWarp0) {
         // ------------------------------------------------------------ unpackers
-        // warps 0-1 of this role widen the 128 A rows, warps 2-3 the 128 B rows;
-        // lane (r, c) = (lane / 4, lane % 4) handles 16 packed bytes of row 8 g + r
-        const int uw = warp - S::kUnpackWarp0;
+        // Group h takes the K steps h, h + kUnpackGroups, ...  Within a group,
+        // A: thread = A row 32 q + lane of TMEM lane quarter q = warp % 4;
+        // B: warp u widens the 8-row groups u, u + 4, ...; lane (r, c) =
+        // (lane / 4, lane % 4) handles 16 packed bytes of row 8 g + r.
+        const int uw = (warp - S::kUnpackWarp0) % S::kUnpackWarps;
+        const int ugroup = (warp - S::kUnpackWarp0) / S::kUnpackWarps;
+        const int q = warp & 3;
+        const int ra = 32 * q + lane;
+        const int aswz = (ra >> 1) & 3;                    // 64-byte swizzle of packed row ra
         const int rsub = lane >> 2;
         const int csub = lane & 3;
-        const int row0 = 8 * S::kGroupsPerWarp * uw;           // 0, 64 (A) or 128, 192 (B)
-        const bool isA = row0 < S::kRows;
-        const int tile_row0 = isA ? row0 : row0 - S::kRows;
-        const uint32_t p_off = isA ? 0u : (uint32_t)S::kPackedA;
-        const uint32_t i_off = isA ? 0u : (uint32_t)S::kABytes;
-        for (int step = 0; step < total; ++step) {
+        const uint32_t a_lane = tmem_base + ((uint32_t)(32 * q) << 16) + S::kACol0;
+        for (int step = ugroup; step < total; step += S::kUnpackGroups) {
             const int ps = step % S::kPStages;
-            const int is = step % S::kIStages;
-            if (!gemm_wait(bar_pfull + 8 * ps, (uint32_t)(step / S::kPStages) & 1, abort_flag))
+            const int bs = step % S::kBStages;
+            const int as = step % S::kAStages;
+            if (!gemm_wait_warp(bar_pfull + 8 * ps, (uint32_t)(step / S::kPStages) & 1, abort_flag))
                 break;
-            uint4 w[S::kGroupsPerWarp];
-            const uint8_t *src = smem + ps * S::kPackedStage + p_off;
+            const uint8_t *src = smem + ps * S::kPackedStage;
+            uint4 wa[4];
 #pragma unroll
-            for (int j = 0; j < S::kGroupsPerWarp; ++j) {
-                const int r = tile_row0 + 8 * j + rsub;
-                w[j] = *reinterpret_cast<const uint4 *>(src + r * (kGemmBK / 2) + csub * 16);
+            for (int c = 0; c < 4; ++c)
+                wa[c] = *reinterpret_cast<const uint4 *>(src + ra * (kGemmBK / 2) + ((c ^ aswz) << 4));
+            uint4 wb[S::kBGroupsPerWarp];
+#pragma unroll
+            for (int j = 0; j < S::kBGroupsPerWarp; ++j) {
+                const int g = uw + S::kUnpackWarps * j;
+                if (g < S::kBGroups)
+                    wb[j] = *reinterpret_cast<const uint4 *>(src + S::kPackedA + (8 * g + rsub) * (kGemmBK / 2) +
+                                                             csub * 16);
             }
-            if (!gemm_wait(bar_iempty + 8 * is, ((uint32_t)(step / S::kIStages) & 1) ^ 1, abort_flag))
+            // A row: packed word i of chunk c holds codes 32 c + [8 i, 8 i + 8);
+            // column 8 c + i gets their low nibbles, column 8 c + 4 + i the high
+            // ones -- the order the B stage uses within each 32-wide K chunk
+            uint32_t av[32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint32_t w4[4] = {wa[c].x, wa[c].y, wa[c].z, wa[c].w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    av[8 * c + i] = (w4[i] << 4) & 0xF0F0F0F0u;
+                    av[8 * c + 4 + i] = w4[i] & 0xF0F0F0F0u;
+                }
+            }
+            // B stage bs is free once the MMAs of step - kBStages are done
+            if (!gemm_wait_warp(bar_sdone + 8 * bs, ((uint32_t)(step / S::kBStages) & 1) ^ 1, abort_flag))
                 break;
-            uint8_t *st_base = smem + S::kIntOffset + is * S::kStageBytes + i_off;
+            uint8_t *st_base = smem + S::kIntOffset + bs * S::kBBytes;
 #pragma unroll
-            for (int j = 0; j < S::kGroupsPerWarp; ++j) {
-                const int r = tile_row0 + 8 * j + rsub;
-                uint8_t *dst = st_base + (r >> 3) * 1024 + (r & 7) * 128;
-                const int sw = r & 7;
-                const uint4 v = w[j];
-                const uint4 lo = make_uint4((v.x << 4) & 0xF0F0F0F0u, (v.y << 4) & 0xF0F0F0F0u,
-                                            (v.z << 4) & 0xF0F0F0F0u, (v.w << 4) & 0xF0F0F0F0u);
-                const uint4 hi = make_uint4(v.x & 0xF0F0F0F0u, v.y & 0xF0F0F0F0u,
-                                            v.z & 0xF0F0F0F0u, v.w & 0xF0F0F0F0u);
-                *reinterpret_cast<uint4 *>(dst + (((2 * csub) ^ sw) << 4)) = lo;
-                *reinterpret_cast<uint4 *>(dst + (((2 * csub + 1) ^ sw) << 4)) = hi;
+            for (int j = 0; j < S::kBGroupsPerWarp; ++j) {
+                const int g = uw + S::kUnpackWarps * j;
+                if (g < S::kBGroups) {
+                    const int r = 8 * g + rsub;
+                    uint8_t *dst = st_base + g * 1024 + rsub * 128;
+                    const uint4 v = wb[j];
+                    const uint4 lo = make_uint4((v.x << 4) & 0xF0F0F0F0u, (v.y << 4) & 0xF0F0F0F0u,
+                                                (v.z << 4) & 0xF0F0F0F0u, (v.w << 4) & 0xF0F0F0F0u);
+                    const uint4 hi = make_uint4(v.x & 0xF0F0F0F0u, v.y & 0xF0F0F0F0u, v.z & 0xF0F0F0F0u,
+                                                v.w & 0xF0F0F0F0u);
+                    *reinterpret_cast<uint4 *>(dst + (((2 * csub) ^ (r & 7)) << 4)) = lo;
+                    *reinterpret_cast<uint4 *>(dst + (((2 * csub + 1) ^ (r & 7)) << 4)) = hi;
+                }
             }
-            // the int8 stage is complete and visible to the tensor core; the
-            // packed stage's reads are complete (their values were stored)
             fence_proxy_async_smem();
-            mbar_arrive_remote(mapa_shared(bar_ifull + 8 * is, 0));
-            mbar_arrive(bar_pempty + 8 * ps);
+            // A stage as is free once the MMAs of step - kAStages are done (MMAs
+            // complete in order, so that step's "done" barrier says so); this
+            // wait is the only one on the tensor core's critical path, and only
+            // the tensor-memory store follows it
+            if (step >= S::kAStages) {
+                const int prev = step - S::kAStages;
+                if (!gemm_wait_warp(bar_sdone + 8 * (prev % S::kBStages), (uint32_t)(prev / S::kBStages) & 1,
+                                    abort_flag))
+                    break;
+            }
+            tc_fence_after();
+            tmem_st32(a_lane + (uint32_t)(32 * as), av);
+            // every lane's part of the int8 stage is complete and visible to the
+            // tensor core, and every value read from the packed stage has been
+            // consumed by a store; the warp barrier orders all lanes' writes
+            // before lane 0's arrivals
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive_remote(mapa_shared(bar_ifull + 8 * bs, 0));
+                mbar_arrive(bar_pempty + 8 * ps);
+            }
         }
     } else if (warp == S::kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer (leader only)
         if (leader && lane == 0) {
-            constexpr uint32_t idesc = idesc_i8(kPairBM, kPairBN);
+            constexpr uint32_t idesc = idesc_i8(kPairBM, BN);
             bool ok = true;
             int step = 0;
             for (int lt = 0; lt < my_tiles && ok; ++lt) {
@@ -202,21 +278,21 @@ int4_gemm_pair_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_
                 if (!gemm_wait(bar_acce + 8 * ab, ((uint32_t)(lt >> 1) & 1) ^ 1, abort_flag))
                     break;
                 tc_fence_after();
-                const uint32_t d = tmem_base + ab * kPairBN;
+                const uint32_t d = tmem_base + ab * BN;
                 for (int kb = 0; kb < KB; ++kb, ++step) {
-                    const int is = step % S::kIStages;
-                    if (!gemm_wait(bar_ifull + 8 * is, (uint32_t)(step / S::kIStages) & 1, abort_flag)) {
+                    const int bsi = step % S::kBStages;
+                    if (!gemm_wait(bar_ifull + 8 * bsi, (uint32_t)(step / S::kBStages) & 1, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t as = sbase + S::kIntOffset + is * S::kStageBytes;
-                    const uint32_t bs = as + S::kABytes;
+                    const uint32_t at = tmem_base + S::kACol0 + 32 * (step % S::kAStages);
+                    const uint32_t bs = sbase + S::kIntOffset + bsi * S::kBBytes;
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
-                        umma_i8_ss_pair(d, desc_kmajor_sw128(as + 32 * j), desc_kmajor_sw128(bs + 32 * j), idesc,
+                        umma_i8_ts_pair(d, at + 8 * j, desc_kmajor_sw128(bs + 32 * j), idesc,
                                         (kb > 0 || j > 0) ? 1u : 0u);
-                    umma_commit_pair(bar_iempty + 8 * is, 0x3);
+                    umma_commit_pair(bar_sdone + 8 * bsi, 0x3);
                     if (kb == KB - 1)
                         umma_commit_pair(bar_accf + 8 * ab, 0x3);
                 }
@@ -232,23 +308,23 @@ int4_gemm_pair_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_
         for (int lt = 0; lt < my_tiles; ++lt) {
             int mb, nb;
             gemm_tile_coords(cluster + lt * nclusters, a.tiles_m, a.tiles_n, mb, nb);
-            const int64_t m = (int64_t)mb * kPairBM + S::kRows * rank + 32 * wq + lane;
-            const int64_t n0 = (int64_t)nb * kPairBN;
+            const int64_t m = (int64_t)mb * kPairBM + S::kRowsA * rank + 32 * wq + lane;
+            const int64_t n0 = (int64_t)nb * BN;
             const bool mrow = m < a.M;
             const int ab = lt & 1;
-            if (!gemm_wait(bar_accf + 8 * ab, (uint32_t)(lt >> 1) & 1, abort_flag))
+            if (!gemm_wait_warp(bar_accf + 8 * ab, (uint32_t)(lt >> 1) & 1, abort_flag))
                 break;
             tc_fence_after();
             float sam = 0.f;
             if (EPI == kEpiScaledF16 && mrow)
                 sam = reinterpret_cast<const float *>(a.sa)[m] * (1.0f / 256.0f);
 #pragma unroll 1
-            for (int c = 0; c < kPairBN / 32; ++c) {
+            for (int c = 0; c < BN / 32; ++c) {
                 uint32_t r[32];
                 __syncwarp();
-                tmem_ld32(lane_addr + ab * kPairBN + 32 * c, r);
+                tmem_ld32(lane_addr + ab * BN + 32 * c, r);
                 tmem_wait_ld(r);
-                if (c == kPairBN / 32 - 1) {
+                if (c == BN / 32 - 1) {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0)

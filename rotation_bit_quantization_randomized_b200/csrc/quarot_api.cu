@@ -263,7 +263,10 @@ quarot_status_t encode_tiled_fn(EncodeTiledFn &fn)
 
 // Tensor map of a packed INT4 matrix [rows, K/2] bytes read in boxes of
 // 64 bytes (128 codes) x box_rows rows; rows past the end read as zeros.
-quarot_status_t packed_map(CUtensorMap &map, const uint8_t *base, int64_t rows, int64_t K, int box_rows)
+// With the 64-byte swizzle the 16-byte chunk c of box row r lands at chunk
+// c ^ ((r / 2) % 4) of that row in shared memory.
+quarot_status_t packed_map(CUtensorMap &map, const uint8_t *base, int64_t rows, int64_t K, int box_rows,
+                           CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE)
 {
     EncodeTiledFn fn;
     quarot_status_t s = encode_tiled_fn(fn);
@@ -274,7 +277,7 @@ quarot_status_t packed_map(CUtensorMap &map, const uint8_t *base, int64_t rows, 
     const cuuint32_t box[2] = {(cuuint32_t)(kGemmBK / 2), (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS)
         return fail(QUAROT_ERR_CUDA, "cuTensorMapEncodeTiled failed (code " + std::to_string((int)r) + ")");
@@ -328,17 +331,21 @@ quarot_status_t launch_gemm(GemmArgs a, cudaStream_t st, bool pdl)
     return after_launch("int4_gemm_kernel launch");
 }
 
+// N tile of the pair GEMM: two accumulator buffers of 224 columns leave
+// tensor memory for two A stages.
+constexpr int kPairBN = 224;
+
 // The per-token / per-channel GEMM on CTA pairs (clusters of two).
 template <int EPI>
 quarot_status_t launch_gemm_pair(GemmArgs a, cudaStream_t st, bool pdl)
 {
-    using S = PairShape<EPI>;
+    using S = PairShape<kPairBN, EPI>;
     int dev;
     DeviceInfo *info;
     quarot_status_t s = current_device(dev, info);
     if (s != QUAROT_OK)
         return s;
-    auto kern = int4_gemm_pair_kernel<EPI>;
+    auto kern = int4_gemm_pair_kernel<kPairBN, EPI>;
     int per_sm = 0;
     s = kernel_occupancy(kern, dev, S::kThreads, S::kSmemBytes, per_sm);
     if (s != QUAROT_OK)
@@ -350,10 +357,10 @@ quarot_status_t launch_gemm_pair(GemmArgs a, cudaStream_t st, bool pdl)
     if (tiles > 0x7fffffff)
         return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "too many output tiles");
     CUtensorMap map_a, map_b;
-    s = packed_map(map_a, a.qa, a.M, a.K, S::kRows);
+    s = packed_map(map_a, a.qa, a.M, a.K, S::kRowsA, CU_TENSOR_MAP_SWIZZLE_64B);
     if (s != QUAROT_OK)
         return s;
-    s = packed_map(map_b, a.qw, a.N, a.K, S::kRows);
+    s = packed_map(map_b, a.qw, a.N, a.K, S::kRowsB);
     if (s != QUAROT_OK)
         return s;
     const int clusters = (int)std::min<int64_t>(tiles, (int64_t)(info->sm_count / 2));

@@ -33,7 +33,7 @@ def _ok(q):
 
 
 S32_SHAPES = [(128, 256, 128), (1, 8, 128), (200, 264, 384), (300, 520, 1024), (129, 256, 8192),
-              (257, 1000, 256), (64, 4096, 512)]
+              (257, 1000, 256), (64, 4096, 512), (4500, 2248, 128)]
 
 
 @pytest.mark.parametrize("M,N,K", S32_SHAPES)
