@@ -41,6 +41,8 @@ def lib():
             "qo_rotate_dense": [P, I64, I64, P, I64, P],
             "qo_quantize": [P, I64, I64, I64, P, P, P],
             "qo_quantize_with_scales": [P, I64, I64, I64, P, P],
+            "qo_quantize_bits": [P, I64, I64, ctypes.c_int, P, P],
+            "qo_quantize_bits_with_scales": [P, I64, I64, ctypes.c_int, P, P],
             "qo_pack": [P, I64, P],
             "qo_unpack": [P, I64, P],
             "qo_int_gemm": [P, P, I64, I64, I64, I64, P],
@@ -157,6 +159,45 @@ def quantize_with_scales(xr, scales, group: int = 0) -> np.ndarray:
     codes = np.empty((M, K), np.int8)
     _check(lib().qo_quantize_with_scales(_p(xr), M, K, group, _p(sc), _p(codes)), "quantize_with_scales")
     return codes
+
+
+def quantize_bits(xr, bits: int):
+    """Per-row symmetric RTN at `bits` bits: (codes int8 [M, K], scales fp64 [M]),
+    s = max|row| / (2^(bits-1) - 1)."""
+    xr = _c(xr, np.float64)
+    M, K = xr.shape
+    codes = np.empty((M, K), np.int8)
+    sc = np.empty((M,), np.float64)
+    _check(lib().qo_quantize_bits(_p(xr), M, K, bits, _p(codes), _p(sc)), "quantize_bits")
+    return codes, sc
+
+
+def quantize_bits_with_scales(xr, scales, bits: int) -> np.ndarray:
+    """RTN codes at `bits` bits of xr [M, K] under given per-row fp64 scales."""
+    xr = _c(xr, np.float64)
+    M, K = xr.shape
+    sc = _c(scales_to_f64(scales), np.float64)
+    codes = np.empty((M, K), np.int8)
+    _check(lib().qo_quantize_bits_with_scales(_p(xr), M, K, bits, _p(sc), _p(codes)), "quantize_bits_with_scales")
+    return codes
+
+
+def rotate_quant8(x16, signs, had_block: int = 0):
+    """The INT8 activation step: rotate, then per-row RTN at 8 bits (codes stay
+    one byte each).  Returns (codes int8 [M, K], scales fp64 [M], x')."""
+    xr = rotate(x16, signs, had_block)
+    codes, sc = quantize_bits(xr, 8)
+    return codes, sc, xr
+
+
+def linear8(x16, w16, signs, had_block: int = 0):
+    """The INT8 prefill linear: both operands rotated and quantized per row at
+    8 bits, then the integer product and the dequantized fp16 output."""
+    qa, sa, _ = rotate_quant8(x16, signs, had_block)
+    qw, sw, _ = rotate_quant8(w16, signs, had_block)
+    acc = int_gemm(qa, qw, 0)
+    y, y16 = dequant_linear(acc, sa, sw, 0)
+    return dict(qa=qa, sa=sa, qw=qw, sw=sw, acc=acc, y=y, y16=y16)
 
 
 def pack(codes) -> np.ndarray:

@@ -297,6 +297,63 @@ int qo_quantize_with_scales(const double *xr, int64_t M, int64_t K, int64_t grou
     return 0;
 }
 
+/* ------------------------------------------------------------------------ */
+/* The same symmetric RTN at other code widths (QuaRot abstract: 4-bit is the */
+/* headline, higher widths are the lossless end of the same recipe; QuaRot    */
+/* summary, "Key points": round-to-nearest without calibration).              */
+/* ------------------------------------------------------------------------ */
+
+/* q = clamp(rint(v / s), -2^(bits-1), 2^(bits-1) - 1); zero scale -> zero. */
+static int32_t rtn_code_bits(double v, double s, int bits)
+{
+    const double qmax = (double)((1 << (bits - 1)) - 1);
+    if (s == 0.0)
+        return 0;
+    double q = nearbyint(v / s);      /* ties to even */
+    if (q < -qmax - 1.0)
+        q = -qmax - 1.0;
+    if (q > qmax)
+        q = qmax;
+    return (int32_t)q;
+}
+
+/*
+ * Per-row symmetric RTN at `bits` (2..8) bits: s = max|row| / (2^(bits-1) - 1)
+ * kept in fp64 (scale64[M]), codes as above, one int8 per element.
+ */
+int qo_quantize_bits(const double *xr, int64_t M, int64_t K, int bits, int8_t *codes, double *scale64)
+{
+    if (M < 0 || K <= 0 || bits < 2 || bits > 8)
+        return -1;
+    const double qmax = (double)((1 << (bits - 1)) - 1);
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; ++r) {
+        const double *v = xr + r * K;
+        double amax = 0.0;
+        for (int64_t k = 0; k < K; ++k)
+            if (fabs(v[k]) > amax)
+                amax = fabs(v[k]);
+        const double s = amax / qmax;
+        scale64[r] = s;
+        for (int64_t k = 0; k < K; ++k)
+            codes[r * K + k] = (int8_t)rtn_code_bits(v[k], s, bits);
+    }
+    return 0;
+}
+
+/* The RTN step alone at `bits` bits with one caller-supplied scale per row. */
+int qo_quantize_bits_with_scales(const double *xr, int64_t M, int64_t K, int bits, const double *scales,
+                                 int8_t *codes)
+{
+    if (M < 0 || K <= 0 || bits < 2 || bits > 8)
+        return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; ++r)
+        for (int64_t k = 0; k < K; ++k)
+            codes[r * K + k] = (int8_t)rtn_code_bits(xr[r * K + k], scales[r], bits);
+    return 0;
+}
+
 /* Nibble packing: byte i = code[2i] in bits 0-3, code[2i+1] in bits 4-7. */
 int qo_pack(const int8_t *codes, int64_t n, uint8_t *packed)
 {
