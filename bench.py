@@ -46,7 +46,8 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--cpu-rows", type=int, default=2048, help="token rows of the CPU-baseline sample")
-    p.add_argument("--case", choices=["gemm", "gemm_group", "rotate", "block", "kvquant", "kvscores"],
+    p.add_argument("--case", choices=["gemm", "gemm_group", "gemm8", "gemm8_full", "rotate", "block", "kvquant",
+                                      "kvscores"],
                    default=None, help="time one kernel on a capture-sized workload (for ncu), not the step")
     return p.parse_args()
 
@@ -404,6 +405,15 @@ def run_case(args):
             sw = torch.rand((N,), device=dev, generator=g) * 1e-3 + 1e-3
         out = torch.empty((M, N), dtype=torch.float16, device=dev)
         fn = lambda: q.quarot_int4_linear(qa, sa, qw, sw, group, out)
+        work, unit = 2.0 * M * N * K / 1e12, "TOPS"
+    elif args.case in ("gemm8", "gemm8_full"):
+        M, N, K = (4096 if args.case == "gemm8" else 32768), 28672, 8192
+        qa = torch.randint(-128, 128, (M, K), dtype=torch.int8, device=dev, generator=g)
+        qw = torch.randint(-128, 128, (N, K), dtype=torch.int8, device=dev, generator=g)
+        sa = torch.rand((M,), device=dev, generator=g) + 0.5
+        sw = torch.rand((N,), device=dev, generator=g) * 1e-5 + 1e-5
+        out = torch.empty((M, N), dtype=torch.float16, device=dev)
+        fn = lambda: q.quarot_int8_linear(qa, sa, qw, sw, out)
         work, unit = 2.0 * M * N * K / 1e12, "TOPS"
     elif args.case in ("rotate", "block"):
         M, K = (8192, 8192) if args.case == "rotate" else (8192, 11008)

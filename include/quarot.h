@@ -185,6 +185,74 @@ quarot_status_t quarot_rotate_quant_linear_noalloc(const void *x_f16, int64_t M,
                                                    void *out_f16, quarot_stream_t stream);
 
 /*
+ * ---------------------------------------------------------------------------
+ * The 8-bit variant of the same recipe: symmetric round-to-nearest codes of
+ * one signed byte each, one scale per row [QR-A: 4-bit is the headline, the
+ * same rotation makes higher widths lossless; QR-S Key points: round-to-
+ * nearest without calibration].  The rotation is the one of
+ * quarot_rotate_quant; only the code width changes:
+ *
+ *   s[m] = max_k |x'[m,k]| / 127 (fp32),  q = rint(x'/s)  (in [-127, 127];
+ *   round half to even; a zero scale gives zero codes)
+ *
+ * INT8 codes are stored one per byte, two's complement, row-major [rows, K].
+ * ---------------------------------------------------------------------------
+ */
+
+/*
+ * quarot_rotate_quant_i8 -- online rotation + 8-bit RTN of activations (or,
+ * offline, of weight rows).  x_f16, signs, had_block, M, K: as in
+ * quarot_rotate_quant (same limits).  q: [M, K] int8 output.  scales: fp32
+ * [M] output.  M == 0 launches nothing and returns QUAROT_OK.
+ */
+quarot_status_t quarot_rotate_quant_i8(const void *x_f16, int64_t M, int64_t K, const int8_t *signs,
+                                       int had_block, int8_t *q, float *scales, quarot_stream_t stream);
+
+/*
+ * quarot_int8_linear -- INT8 x INT8 linear layer, int32 accumulation on the
+ * tensor cores, fused dequantizing epilogue [QR-S Summary: products in
+ * integers]:
+ *   out[m,n] = fp16( acc[m,n] * s_a[m] * s_w[n] ),  acc = sum_k qa[m,k] qw[n,k]
+ * (exact: |acc| <= 2^14 K < 2^31).
+ * qa [M, K] int8, s_a fp32 [M]; qw [N, K] int8 (rows rotated with the same
+ * signs and Hadamard [DQ-1]), s_w fp32 [N]; out [M, N] fp16.
+ * Limits: M >= 0 (0 launches nothing), N >= 1 with N % 8 == 0,
+ *         K % 128 == 0 with 128 <= K <= 65536.
+ */
+quarot_status_t quarot_int8_linear(const int8_t *qa, const float *s_a, int64_t M, const int8_t *qw,
+                                   const float *s_w, int64_t N, int64_t K, void *out_f16,
+                                   quarot_stream_t stream);
+
+/*
+ * quarot_int8_gemm_s32 -- the same integer product without the epilogue,
+ * acc[m,n] written as int32 [M, N]; exact for every input.  Layouts and
+ * limits as quarot_int8_linear (no scales).
+ */
+quarot_status_t quarot_int8_gemm_s32(const int8_t *qa, int64_t M, const int8_t *qw, int64_t N, int64_t K,
+                                     int32_t *acc, quarot_stream_t stream);
+
+/*
+ * quarot_rotate_quant_linear_i8_workspace -- bytes of device workspace that
+ * quarot_rotate_quant_linear_i8 needs: the INT8 activation codes [M, K] and
+ * their fp32 scales, each at a 256-byte aligned offset.
+ */
+size_t quarot_rotate_quant_linear_i8_workspace(int64_t M, int64_t K);
+
+/*
+ * quarot_rotate_quant_linear_i8 -- the fused online path of one INT8 linear
+ * layer: quarot_rotate_quant_i8 of x into `workspace`, then
+ * quarot_int8_linear against the prepared weights, both on `stream` (the
+ * GEMM launched as a programmatic dependent of the quantizer).  Arguments as
+ * in those calls; workspace: caller-owned device memory of at least
+ * quarot_rotate_quant_linear_i8_workspace(M, K) bytes, 256-byte aligned,
+ * scratch; ws_bytes: its size.
+ */
+quarot_status_t quarot_rotate_quant_linear_i8(const void *x_f16, int64_t M, int64_t K, const int8_t *signs,
+                                              int had_block, const int8_t *qw, const float *s_w, int64_t N,
+                                              void *workspace, size_t ws_bytes, void *out_f16,
+                                              quarot_stream_t stream);
+
+/*
  * quarot_kv_quant -- INT4 KV-cache write [QR-A: the KV cache in 4 bits;
  * DQ-12: fixed Hadamard on the query-key product, per-head quantization].
  *

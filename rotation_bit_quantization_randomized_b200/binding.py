@@ -35,6 +35,11 @@ _SIGS = {
     "quarot_rotate_quant_linear_workspace": ([_I64, _I64, _INT], _SZ),
     "quarot_rotate_quant_linear": ([_P, _I64, _I64, _P, _INT, _INT, _P, _P, _I64, _P, _SZ, _P, _P], _INT),
     "quarot_rotate_quant_linear_noalloc": ([_P, _I64, _I64, _P, _INT, _INT, _P, _P, _I64, _P, _P], _INT),
+    "quarot_rotate_quant_i8": ([_P, _I64, _I64, _P, _INT, _P, _P, _P], _INT),
+    "quarot_int8_linear": ([_P, _P, _I64, _P, _P, _I64, _I64, _P, _P], _INT),
+    "quarot_int8_gemm_s32": ([_P, _I64, _P, _I64, _I64, _P, _P], _INT),
+    "quarot_rotate_quant_linear_i8_workspace": ([_I64, _I64], _SZ),
+    "quarot_rotate_quant_linear_i8": ([_P, _I64, _I64, _P, _INT, _P, _P, _I64, _P, _SZ, _P, _P], _INT),
     "quarot_kv_quant": ([_P, _P, _I64, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P], _INT),
     "quarot_kv_decode_scores": ([_P, _I64, _I64, _P, _P, _P, _I64, _I64, _I64, _P, _P], _INT),
     "quarot_get_device_status": ([], _INT),
@@ -167,6 +172,65 @@ def quarot_rotate_quant_linear_noalloc(x: torch.Tensor, signs: torch.Tensor, qw:
     _check("quarot_rotate_quant_linear_noalloc",
            lib.quarot_rotate_quant_linear_noalloc(_ptr(x), M, K, _ptr(signs), had_block, group, _ptr(qw),
                                                   _ptr(s_w), N, _ptr(out), _stream(stream)))
+    return out
+
+
+def quarot_rotate_quant_i8(x: torch.Tensor, signs: torch.Tensor, had_block: int = 0,
+                           q: Optional[torch.Tensor] = None, scales: Optional[torch.Tensor] = None, stream=None):
+    """x fp16 [M, K] -> (q int8 [M, K], scales fp32 [M]): the 8-bit variant."""
+    M, K = x.shape
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if scales is None:
+        scales = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _check("quarot_rotate_quant_i8",
+           lib.quarot_rotate_quant_i8(_ptr(x), M, K, _ptr(signs), had_block, _ptr(q), _ptr(scales),
+                                      _stream(stream)))
+    return q, scales
+
+
+def quarot_int8_linear(qa: torch.Tensor, s_a: torch.Tensor, qw: torch.Tensor, s_w: torch.Tensor,
+                       out: Optional[torch.Tensor] = None, stream=None):
+    """INT8 [M, K] x INT8 [N, K]^T with fp32 scales -> fp16 [M, N]."""
+    M, K = qa.shape
+    N = qw.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=qa.device)
+    _check("quarot_int8_linear",
+           lib.quarot_int8_linear(_ptr(qa), _ptr(s_a), M, _ptr(qw), _ptr(s_w), N, K, _ptr(out), _stream(stream)))
+    return out
+
+
+def quarot_int8_gemm_s32(qa: torch.Tensor, qw: torch.Tensor, acc: Optional[torch.Tensor] = None, stream=None):
+    """Exact int32 [M, N] = qa . qw^T for int8 codes."""
+    M, K = qa.shape
+    N = qw.shape[0]
+    if acc is None:
+        acc = torch.empty((M, N), dtype=torch.int32, device=qa.device)
+    _check("quarot_int8_gemm_s32",
+           lib.quarot_int8_gemm_s32(_ptr(qa), M, _ptr(qw), N, K, _ptr(acc), _stream(stream)))
+    return acc
+
+
+def quarot_rotate_quant_linear_i8_workspace(M: int, K: int) -> int:
+    return int(lib.quarot_rotate_quant_linear_i8_workspace(M, K))
+
+
+def quarot_rotate_quant_linear_i8(x: torch.Tensor, signs: torch.Tensor, qw: torch.Tensor, s_w: torch.Tensor,
+                                  had_block: int = 0, workspace: Optional[torch.Tensor] = None,
+                                  out: Optional[torch.Tensor] = None, stream=None):
+    """Fused online INT8 path: rotate + 8-bit quantize x, then the INT8 linear; fp16 [M, N]."""
+    M, K = x.shape
+    N = qw.shape[0]
+    need = quarot_rotate_quant_linear_i8_workspace(M, K)
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=x.device)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=x.device)
+    _check("quarot_rotate_quant_linear_i8",
+           lib.quarot_rotate_quant_linear_i8(_ptr(x), M, K, _ptr(signs), had_block, _ptr(qw), _ptr(s_w), N,
+                                             _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                             _ptr(out), _stream(stream)))
     return out
 
 

@@ -6,6 +6,7 @@
 #include "common.cuh"
 #include "int4_gemm.cuh"
 #include "int4_gemm_pair.cuh"
+#include "int8_gemm_pair.cuh"
 #include "kv_scores.cuh"
 #include "rotate_quant.cuh"
 
@@ -144,11 +145,14 @@ quarot_status_t check_rotate_args(const void *x, int64_t M, int64_t K, const int
     return QUAROT_OK;
 }
 
-template <int LOGN, int GROUP>
+// qmax of a code width: the largest code magnitude of the symmetric RTN.
+constexpr double qmax_of(int bits) { return bits == 8 ? 127.0 : 7.0; }
+
+template <int LOGN, int GROUP, int BITS>
 quarot_status_t launch_fwht(const void *x, int64_t M, const int8_t *signs, uint8_t *q, void *scales,
                             cudaStream_t st, int dev, int sms)
 {
-    auto kern = fwht_quant_kernel<LOGN, GROUP>;
+    auto kern = fwht_quant_kernel<LOGN, GROUP, BITS>;
     int per_sm = 0;
     quarot_status_t s = kernel_occupancy(kern, dev, kFwhtThreads, 0, per_sm);
     if (s != QUAROT_OK)
@@ -158,32 +162,33 @@ quarot_status_t launch_fwht(const void *x, int64_t M, const int8_t *signs, uint8
     const int grid = (int)std::min<int64_t>(ctas, (int64_t)sms * per_sm);
     const double n = double(1 << LOGN);
     kern<<<grid, kFwhtThreads, 0, st>>>(reinterpret_cast<const uint32_t *>(x), M, signs, q, scales,
-                                        (float)(1.0 / (7.0 * std::sqrt(n))), (float)std::sqrt(n));
+                                        (float)(1.0 / (qmax_of(BITS) * std::sqrt(n))), (float)std::sqrt(n));
     return after_launch("fwht_quant_kernel launch");
 }
 
-template <int GROUP>
+template <int GROUP, int BITS>
 quarot_status_t dispatch_fwht(int logn, const void *x, int64_t M, const int8_t *signs, uint8_t *q,
                               void *scales, cudaStream_t st, int dev, int sms)
 {
     switch (logn) {
-    case 8: return launch_fwht<8, GROUP>(x, M, signs, q, scales, st, dev, sms);
-    case 9: return launch_fwht<9, GROUP>(x, M, signs, q, scales, st, dev, sms);
-    case 10: return launch_fwht<10, GROUP>(x, M, signs, q, scales, st, dev, sms);
-    case 11: return launch_fwht<11, GROUP>(x, M, signs, q, scales, st, dev, sms);
-    case 12: return launch_fwht<12, GROUP>(x, M, signs, q, scales, st, dev, sms);
-    case 13: return launch_fwht<13, GROUP>(x, M, signs, q, scales, st, dev, sms);
+    case 8: return launch_fwht<8, GROUP, BITS>(x, M, signs, q, scales, st, dev, sms);
+    case 9: return launch_fwht<9, GROUP, BITS>(x, M, signs, q, scales, st, dev, sms);
+    case 10: return launch_fwht<10, GROUP, BITS>(x, M, signs, q, scales, st, dev, sms);
+    case 11: return launch_fwht<11, GROUP, BITS>(x, M, signs, q, scales, st, dev, sms);
+    case 12: return launch_fwht<12, GROUP, BITS>(x, M, signs, q, scales, st, dev, sms);
+    case 13: return launch_fwht<13, GROUP, BITS>(x, M, signs, q, scales, st, dev, sms);
     default: return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "unsupported transform size");
     }
 }
 
-template <bool ROTATE, int GROUP>
+template <bool ROTATE, int GROUP, int BITS = 4>
 quarot_status_t launch_block(const void *x, int64_t M, int64_t K, const int8_t *signs, uint8_t *q,
                              void *scales, float scale_mul, float sqrt_n, cudaStream_t st, int dev, int sms)
 {
     const int nb = (int)(K / 128);
     const bool multi = nb > kBlockThreads;
-    auto kern = multi ? block128_quant_kernel<ROTATE, GROUP, true> : block128_quant_kernel<ROTATE, GROUP, false>;
+    auto kern = multi ? block128_quant_kernel<ROTATE, GROUP, true, BITS>
+                      : block128_quant_kernel<ROTATE, GROUP, false, BITS>;
     const int rows_per_cta = multi ? 1 : kBlockThreads / nb;
     const int threads = multi ? kBlockThreads : ((rows_per_cta * nb + 31) / 32) * 32;
     int per_sm = 0;
@@ -197,23 +202,29 @@ quarot_status_t launch_block(const void *x, int64_t M, int64_t K, const int8_t *
     return after_launch("block128_quant_kernel launch");
 }
 
+// bits == 8 implies group == 0 (checked by the callers).
 quarot_status_t rotate_quant_launch(const void *x, int64_t M, int64_t K, const int8_t *signs, int had_block,
-                                    int group, uint8_t *q, void *scales, cudaStream_t st)
+                                    int group, uint8_t *q, void *scales, cudaStream_t st, int bits = 4)
 {
     int dev;
     DeviceInfo *info;
     quarot_status_t s = current_device(dev, info);
     if (s != QUAROT_OK)
         return s;
+    const int sms = info->sm_count;
     if (had_block == 0 && K >= 256) {
         const int logn = ilog2(K);
-        return group == 0 ? dispatch_fwht<0>(logn, x, M, signs, q, scales, st, dev, info->sm_count)
-                          : dispatch_fwht<128>(logn, x, M, signs, q, scales, st, dev, info->sm_count);
+        if (bits == 8)
+            return dispatch_fwht<0, 8>(logn, x, M, signs, q, scales, st, dev, sms);
+        return group == 0 ? dispatch_fwht<0, 4>(logn, x, M, signs, q, scales, st, dev, sms)
+                          : dispatch_fwht<128, 4>(logn, x, M, signs, q, scales, st, dev, sms);
     }
-    const float mul = (float)(1.0 / (7.0 * std::sqrt(128.0)));
+    const float mul = (float)(1.0 / (qmax_of(bits) * std::sqrt(128.0)));
     const float sq = (float)std::sqrt(128.0);
-    return group == 0 ? launch_block<true, 0>(x, M, K, signs, q, scales, mul, sq, st, dev, info->sm_count)
-                      : launch_block<true, 128>(x, M, K, signs, q, scales, mul, sq, st, dev, info->sm_count);
+    if (bits == 8)
+        return launch_block<true, 0, 8>(x, M, K, signs, q, scales, mul, sq, st, dev, sms);
+    return group == 0 ? launch_block<true, 0>(x, M, K, signs, q, scales, mul, sq, st, dev, sms)
+                      : launch_block<true, 128>(x, M, K, signs, q, scales, mul, sq, st, dev, sms);
 }
 
 // ----------------------------------------------------------------- GEMM
@@ -389,6 +400,96 @@ quarot_status_t launch_gemm_pair(GemmArgs a, cudaStream_t st, bool pdl)
     return after_launch("int4_gemm_pair_kernel launch");
 }
 
+// Tensor map of an INT8 code matrix [rows, K] read in boxes of 128 bytes x
+// 128 rows with the 128-byte swizzle -- the K-major layout the MMA reads;
+// rows past the end read as zeros.
+quarot_status_t i8_map(CUtensorMap &map, const int8_t *base, int64_t rows, int64_t K)
+{
+    EncodeTiledFn fn;
+    quarot_status_t s = encode_tiled_fn(fn);
+    if (s != QUAROT_OK)
+        return s;
+    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)K};
+    const cuuint32_t box[2] = {(cuuint32_t)kGemmBK, (cuuint32_t)I8PairShape::kRows};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(QUAROT_ERR_CUDA, "cuTensorMapEncodeTiled failed (code " + std::to_string((int)r) + ")");
+    return QUAROT_OK;
+}
+
+// The INT8 GEMM on CTA pairs (clusters of two); a.qa / a.qw hold int8 codes.
+template <int EPI>
+quarot_status_t launch_gemm_i8(GemmArgs a, cudaStream_t st, bool pdl)
+{
+    using S = I8PairShape;
+    int dev;
+    DeviceInfo *info;
+    quarot_status_t s = current_device(dev, info);
+    if (s != QUAROT_OK)
+        return s;
+    auto kern = int8_gemm_pair_kernel<EPI>;
+    int per_sm = 0;
+    s = kernel_occupancy(kern, dev, S::kThreads, S::kSmemBytes, per_sm);
+    if (s != QUAROT_OK)
+        return s;
+    a.tiles_m = (int)((a.M + kI8PairBM - 1) / kI8PairBM);
+    a.tiles_n = (int)((a.N + kI8PairBN - 1) / kI8PairBN);
+    a.kblocks = (int)(a.K / kGemmBK);
+    const int64_t tiles = (int64_t)a.tiles_m * a.tiles_n;
+    if (tiles > 0x7fffffff)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "too many output tiles");
+    CUtensorMap map_a, map_b;
+    s = i8_map(map_a, reinterpret_cast<const int8_t *>(a.qa), a.M, a.K);
+    if (s != QUAROT_OK)
+        return s;
+    s = i8_map(map_b, reinterpret_cast<const int8_t *>(a.qw), a.N, a.K);
+    if (s != QUAROT_OK)
+        return s;
+    const int clusters = (int)std::min<int64_t>(tiles, (int64_t)(info->sm_count / 2));
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * clusters);
+    cfg.blockDim = dim3(S::kThreads);
+    cfg.dynamicSmemBytes = S::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    int nattr = 1;
+    if (pdl) {
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        nattr = 2;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = nattr;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a, map_a, map_b);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "int8_gemm_pair_kernel launch");
+    return after_launch("int8_gemm_pair_kernel launch");
+}
+
+quarot_status_t linear8_launch(const int8_t *qa, const float *sa, int64_t M, const int8_t *qw, const float *sw,
+                               int64_t N, int64_t K, void *out, cudaStream_t st, bool pdl)
+{
+    GemmArgs a = {};
+    a.qa = reinterpret_cast<const uint8_t *>(qa);
+    a.sa = sa;
+    a.qw = reinterpret_cast<const uint8_t *>(qw);
+    a.sw = sw;
+    a.out = out;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    return launch_gemm_i8<kEpiScaledF16>(a, st, pdl);
+}
+
 quarot_status_t linear_launch(const uint8_t *qa, const void *sa, int64_t M, const uint8_t *qw, const void *sw,
                               int64_t N, int64_t K, int group, void *out, cudaStream_t st, bool pdl)
 {
@@ -536,6 +637,73 @@ quarot_status_t quarot_rotate_quant_linear_noalloc(const void *x_f16, int64_t M,
     if (s != QUAROT_OK)
         return s;
     return linear_launch(qa, sa, M, qw, s_w, N, K, group, out_f16, st, true);
+}
+
+quarot_status_t quarot_rotate_quant_i8(const void *x_f16, int64_t M, int64_t K, const int8_t *signs, int had_block,
+                                       int8_t *q, float *scales, quarot_stream_t stream)
+{
+    quarot_status_t s = check_rotate_args(x_f16, M, K, signs, had_block, 0, q, scales);
+    if (s != QUAROT_OK || M == 0)
+        return s;
+    return rotate_quant_launch(x_f16, M, K, signs, had_block, 0, reinterpret_cast<uint8_t *>(q), scales,
+                               (cudaStream_t)stream, 8);
+}
+
+quarot_status_t quarot_int8_linear(const int8_t *qa, const float *s_a, int64_t M, const int8_t *qw, const float *s_w,
+                                   int64_t N, int64_t K, void *out_f16, quarot_stream_t stream)
+{
+    quarot_status_t s = check_gemm_args(qa, M, qw, N, K, out_f16, s_a, s_w, true);
+    if (s != QUAROT_OK || M == 0)
+        return s;
+    return linear8_launch(qa, s_a, M, qw, s_w, N, K, out_f16, (cudaStream_t)stream, false);
+}
+
+quarot_status_t quarot_int8_gemm_s32(const int8_t *qa, int64_t M, const int8_t *qw, int64_t N, int64_t K,
+                                     int32_t *acc, quarot_stream_t stream)
+{
+    quarot_status_t s = check_gemm_args(qa, M, qw, N, K, acc, nullptr, nullptr, false);
+    if (s != QUAROT_OK || M == 0)
+        return s;
+    GemmArgs a = {};
+    a.qa = reinterpret_cast<const uint8_t *>(qa);
+    a.qw = reinterpret_cast<const uint8_t *>(qw);
+    a.out = acc;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    return launch_gemm_i8<kEpiS32>(a, (cudaStream_t)stream, false);
+}
+
+size_t quarot_rotate_quant_linear_i8_workspace(int64_t M, int64_t K)
+{
+    if (M <= 0 || K <= 0)
+        return 0;
+    return align256((size_t)M * (size_t)K) + align256((size_t)M * 4);
+}
+
+quarot_status_t quarot_rotate_quant_linear_i8(const void *x_f16, int64_t M, int64_t K, const int8_t *signs,
+                                              int had_block, const int8_t *qw, const float *s_w, int64_t N,
+                                              void *workspace, size_t ws_bytes, void *out_f16,
+                                              quarot_stream_t stream)
+{
+    quarot_status_t s = check_rotate_args(x_f16, M, K, signs, had_block, 0, workspace, workspace);
+    if (s != QUAROT_OK)
+        return s;
+    s = check_gemm_args(workspace, M, qw, N, K, out_f16, workspace, s_w, true);
+    if (s != QUAROT_OK || M == 0)
+        return s;
+    const size_t need = quarot_rotate_quant_linear_i8_workspace(M, K);
+    if (ws_bytes < need)
+        return fail(QUAROT_ERR_INVALID_ARG, "workspace too small");
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(QUAROT_ERR_MISALIGNED, "workspace must be 256-byte aligned");
+    int8_t *qa = static_cast<int8_t *>(workspace);
+    float *sa = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + align256((size_t)M * (size_t)K));
+    cudaStream_t st = (cudaStream_t)stream;
+    s = rotate_quant_launch(x_f16, M, K, signs, had_block, 0, reinterpret_cast<uint8_t *>(qa), sa, st, 8);
+    if (s != QUAROT_OK)
+        return s;
+    return linear8_launch(qa, sa, M, qw, s_w, N, K, out_f16, st, true);
 }
 
 quarot_status_t quarot_kv_quant(const void *k_f16, const void *v_f16, int64_t B, int64_t T, int64_t Hkv, int64_t D,

@@ -79,6 +79,30 @@ __device__ __forceinline__ void quant_pack_store(const float (&v)[128], float r,
     }
 }
 
+// Rounds 128 values of one thread to signed 8-bit codes and stores the 128
+// bytes (the 8-bit variant of the same RTN).  r = 127 / max|y| of the row, so
+// |v r| <= 127 (1 + 2^-23) and no clamp is needed; the low byte of the bit
+// pattern of fma(v, r, 1.5 * 2^23) is the two's-complement code.
+__device__ __forceinline__ void quant_store_i8(const float (&v)[128], float r, int8_t *dst, bool valid)
+{
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const int e = 16 * i + 4 * w;
+            float f0, f1, f2, f3;
+            fma_x2(v[e], v[e + 1], r, 12582912.0f, f0, f1);
+            fma_x2(v[e + 2], v[e + 3], r, 12582912.0f, f2, f3);
+            const uint32_t lo = __byte_perm(__float_as_uint(f0), __float_as_uint(f1), 0x0040);
+            const uint32_t hi = __byte_perm(__float_as_uint(f2), __float_as_uint(f3), 0x0040);
+            pk[w] = __byte_perm(lo, hi, 0x5410);
+        }
+        if (valid)
+            reinterpret_cast<uint4 *>(dst)[i] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
+}
+
 // fp16 group scale of a block and the matching code multiplier.
 __device__ __forceinline__ float group_scale(float amax, float scale_mul, float sqrt_n, __half &s16)
 {
@@ -90,16 +114,18 @@ __device__ __forceinline__ float group_scale(float amax, float scale_mul, float 
 // ---------------------------------------------------------------------------
 // Full transform, K = 2^LOGN with 8 <= LOGN <= 13.
 // ---------------------------------------------------------------------------
-template <int LOGN, int GROUP>
+template <int LOGN, int GROUP, int BITS = 4>
 __global__ void __launch_bounds__(kFwhtThreads, 4)
 fwht_quant_kernel(const uint32_t *__restrict__ x,      // [M, K/2] fp16 pairs
                   int64_t M, const int8_t *__restrict__ signs,
-                  uint8_t *__restrict__ q,             // [M, K/2]
+                  uint8_t *__restrict__ q,             // [M, K/2] (4-bit) or [M, K] (8-bit)
                   void *__restrict__ scales,           // fp32 [M] or fp16 [M, K/128]
-                  float scale_mul,                     // 1 / (7 sqrt(K)), rounded to fp32
+                  float scale_mul,                     // 1 / (qmax sqrt(K)), rounded to fp32
                   float sqrt_n)                        // sqrt(K), rounded to fp32
 {
     static_assert(LOGN >= 8 && LOGN <= 13, "full transform covers 256..8192");
+    static_assert(BITS == 4 || (BITS == 8 && GROUP == 0), "8-bit codes use one scale per row");
+    constexpr float kQmax = BITS == 8 ? 127.0f : 7.0f;
     constexpr int N = 1 << LOGN;
     constexpr int T = N / 128;              // threads per row
     constexpr int R = kFwhtThreads / T;     // rows per CTA iteration
@@ -188,7 +214,7 @@ fwht_quant_kernel(const uint32_t *__restrict__ x,      // [M, K/2] fp16 pairs
                 __syncthreads();
                 amax = fmaxf(red[0], red[1]);
             }
-            r = amax > 0.f ? 7.0f / amax : 0.f;
+            r = amax > 0.f ? kQmax / amax : 0.f;
             if (valid && tr == 0)
                 reinterpret_cast<float *>(scales)[row] = amax * scale_mul;
         } else {
@@ -198,7 +224,10 @@ fwht_quant_kernel(const uint32_t *__restrict__ x,      // [M, K/2] fp16 pairs
             if (valid)
                 reinterpret_cast<__half *>(scales)[row * (N / 128) + tr] = s16;
         }
-        quant_pack_store<GROUP>(v, r, q + (valid ? row : 0) * (N / 2) + tr * 64, valid);
+        if (BITS == 8)
+            quant_store_i8(v, r, reinterpret_cast<int8_t *>(q) + (valid ? row : 0) * N + tr * 128, valid);
+        else
+            quant_pack_store<GROUP>(v, r, q + (valid ? row : 0) * (N / 2) + tr * 64, valid);
     }
     // a dependent GEMM launched with programmatic serialization may start now
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -234,14 +263,18 @@ __device__ __forceinline__ void load_block(const uint4 *__restrict__ src, bool v
         fwht_bits<0, 7>(v);
 }
 
-template <bool ROTATE, int GROUP, bool MULTI>
+template <bool ROTATE, int GROUP, bool MULTI, int BITS = 4>
 __global__ void __launch_bounds__(kBlockThreads)
 block128_quant_kernel(const uint4 *__restrict__ x,     // [M, K] fp16, 8 per uint4
                       int64_t M, int K, int rows_per_cta,
                       const int8_t *__restrict__ signs,
-                      uint8_t *__restrict__ q, void *__restrict__ scales,
+                      uint8_t *__restrict__ q,         // [M, K/2] (4-bit) or [M, K] (8-bit)
+                      void *__restrict__ scales,
                       float scale_mul, float sqrt_n)
 {
+    static_assert(BITS == 4 || (BITS == 8 && GROUP == 0), "8-bit codes use one scale per row");
+    constexpr float kQmax = BITS == 8 ? 127.0f : 7.0f;
+    constexpr int kCodeBytes = BITS == 8 ? 128 : 64;   // bytes of one 128-block's codes
     constexpr int BPT = MULTI ? 4 : 1;                 // blocks per thread, at most
     __shared__ unsigned int rowmax[kBlockThreads];
     __shared__ uint32_t sgn_multi[MULTI ? BPT * 4 * kBlockThreads : 1];   // [block i][word][thread]
@@ -280,7 +313,7 @@ block128_quant_kernel(const uint4 *__restrict__ x,     // [M, K] fp16, 8 per uin
         const int64_t row = row0 + rl;
         const bool row_ok = active && row < M;
         const uint4 *xrow = x + (row_ok ? row : 0) * (K / 8);
-        uint8_t *qrow = q + (row_ok ? row : 0) * (K / 2);
+        uint8_t *qrow = q + (row_ok ? row : 0) * ((int64_t)K * BITS / 8);
 
         if (GROUP != 0) {
             // independent blocks
@@ -327,11 +360,17 @@ block128_quant_kernel(const uint4 *__restrict__ x,     // [M, K] fp16, 8 per uin
             __syncthreads();
             amax = active ? __uint_as_float(rowmax[rl]) : 0.f;
             __syncthreads();
-            const float r = amax > 0.f ? 7.0f / amax : 0.f;
+            const float r = amax > 0.f ? kQmax / amax : 0.f;
             if (row_ok && b0 == 0)
                 reinterpret_cast<float *>(scales)[row] = amax * scale_mul;
+            auto store = [&](uint8_t *dst, bool ok) {
+                if (BITS == 8)
+                    quant_store_i8(v, r, reinterpret_cast<int8_t *>(dst), ok);
+                else
+                    quant_pack_store<0>(v, r, dst, ok);
+            };
             if (!MULTI) {
-                quant_pack_store<0>(v, r, qrow + b0 * 64, row_ok);
+                store(qrow + b0 * kCodeBytes, row_ok);
             } else {
 #pragma unroll 1
                 for (int i = 0; i < BPT; ++i) {
@@ -340,7 +379,7 @@ block128_quant_kernel(const uint4 *__restrict__ x,     // [M, K] fp16, 8 per uin
                     uint32_t sg[4];
                     block_signs(i, sg);
                     load_block<ROTATE>(xrow + (ok ? b : 0) * 16, ok, sg, v);
-                    quant_pack_store<0>(v, r, qrow + (ok ? b : 0) * 64, ok);
+                    store(qrow + (ok ? b : 0) * kCodeBytes, ok);
                 }
             }
         }

@@ -100,3 +100,36 @@ def check_f16_output(y_gpu_f16, y_ref, tol=2e-3):
     worst = float(err.max()) if err.size else 0.0
     assert worst <= tol, f"max relative error {worst:.3e} > {tol}"
     return worst
+
+
+def check_codes_bits(gpu_codes, gpu_scales, xr, bits, max_frac=1e-4):
+    """The scale and code rules for per-row codes of `bits` bits stored one per
+    byte (the 8-bit variant): scale within 1e-6 relative of the oracle's fp64
+    max|x'| / (2^(bits-1) - 1); codes equal the oracle's RTN under the device
+    scale, or +-1 only at near-ties (same budget and exact-tie rule as the
+    INT4 check).  Returns the number of flips."""
+    qmax = float((1 << (bits - 1)) - 1)
+    M, K = xr.shape
+    amax = np.abs(xr).max(axis=1)
+    ref = amax / qmax
+    got_s = np.asarray(gpu_scales, np.float64)
+    rel = np.abs(got_s - ref) / np.maximum(ref, 1e-300)
+    bad = (rel > 1e-6) & ~((ref == 0) & (got_s == 0))
+    assert not np.any(bad), f"per-row scales off: max rel {rel[bad].max():.3e}"
+    expect = oracle.quantize_bits_with_scales(xr, got_s, bits)
+    got = np.asarray(gpu_codes).view(np.int8).reshape(M, K)
+    d = got.astype(np.int16) - expect.astype(np.int16)
+    flips = d != 0
+    n = int(flips.sum())
+    if n == 0:
+        return 0
+    assert np.all(np.abs(d[flips]) == 1), "codes differ by more than one step"
+    t = np.where(got_s[:, None] > 0, xr / np.where(got_s[:, None] > 0, got_s[:, None], 1.0), 0.0)
+    dist = np.abs(t - (np.floor(t) + 0.5))
+    assert np.all(dist[flips] < 1e-3), f"code flips away from near-ties (max dist {dist[flips].max():.3e})"
+    s0 = ref[:, None]
+    t0 = np.where(s0 > 0, xr / np.where(s0 > 0, s0, 1.0), 0.0)
+    exact_tie = np.abs(t0 - (np.floor(t0) + 0.5)) <= 1e-9 * np.maximum(1.0, np.abs(t0))
+    counted = int((flips & ~exact_tie).sum())
+    assert counted <= max_frac * got.size, f"{counted} near-tie code flips in {got.size} elements"
+    return n

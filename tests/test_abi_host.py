@@ -107,3 +107,26 @@ def test_binding_raises_on_error(q):
     s = torch.ones(384, dtype=torch.int8)
     with pytest.raises(q.QuarotError, match="UNSUPPORTED_SHAPE"):
         q.quarot_rotate_quant(x, s)
+
+
+def test_int8_entry_points_reject(q):
+    rq8 = q.lib.quarot_rotate_quant_i8
+    assert rq8(A16, 4, 384, A16, 0, A16, A16, None) == 2          # not a power of two
+    assert rq8(A16, 4, 256, A16, 64, A16, A16, None) == 1         # had_block
+    assert rq8(A16, 4, 256, A16, 0, MIS, A16, None) == 3
+    assert rq8(None, 0, 256, None, 0, None, None, None) == 0      # empty: no launch
+    lin8 = q.lib.quarot_int8_linear
+    assert lin8(A16, A16, 4, A16, A16, 100, 256, A16, None) == 2  # N % 8
+    assert lin8(A16, A16, 4, A16, A16, 256, 200, A16, None) == 2  # K % 128
+    assert lin8(A16, None, 4, A16, A16, 256, 256, A16, None) == 1
+    assert lin8(None, None, 0, A16, A16, 256, 256, None, None) == 0
+    s32 = q.lib.quarot_int8_gemm_s32
+    assert s32(A16, 4, A16, 12, 256, A16, None) == 2
+    assert s32(A16, 4, A16, 16, 256, MIS, None) == 3
+    ws = q.lib.quarot_rotate_quant_linear_i8_workspace
+    assert ws(0, 256) == 0
+    assert ws(16, 256) == 4096 + 256                               # int8 codes, then fp32 scales
+    f = q.lib.quarot_rotate_quant_linear_i8
+    need = ws(16, 256)
+    assert f(A16, 16, 256, A16, 0, A16, A16, 256, A16, need - 1, A16, None) == 1
+    assert f(A16, 16, 256, A16, 0, A16, A16, 256, P(0x10010), need, A16, None) == 3
