@@ -22,7 +22,7 @@
 //  * Full transform (n = 2^p, 256 <= n <= 8192): each row is owned by
 //    T = n/128 threads holding 128 values each.  Phase A loads fp16 pairs so
 //    that a thread holds element bit 0 and the top six element bits, and
-//    applies the Walsh-Hadamard along those 7 bits in registers.  A swizzled
+//    applies the Walsh-Hadamard along those 7 bits in registers.  A padded
 //    shared-memory transpose then gives each thread 128 contiguous elements
 //    (bits 0-6) for phase B, which finishes bits 1..min(6, p-7).  Because
 //    H_n = H_2 (x) ... (x) H_2 (Sylvester), stages along different bits
@@ -132,13 +132,19 @@ fwht_quant_kernel(const uint32_t *__restrict__ x,      // [M, K/2] fp16 pairs
     constexpr int SH = LOGN - 6;            // element shift of the phase-A pair index j
     constexpr int PB = (LOGN - 7) < 6 ? (LOGN - 7) : 6;   // phase-B bits 1..PB
 
-    __shared__ __align__(16) float buf[R * N];
+    // transpose buffer: each 128-element chunk padded to 132 floats and each
+    // row of the CTA iteration by 4 more (8 at K = 1024), so that the phase-A
+    // writes of a warp take 2 wavefronts per 256 B and its phase-B reads 4 per
+    // 512 B (the minimum) at every K, and every address is a per-thread base
+    // plus a compile-time offset
+    constexpr int kChunk = 132;
+    constexpr int kRowFloats = (N / 128) * kChunk + (LOGN == 10 ? 8 : 4);
+    __shared__ __align__(16) float buf[R * kRowFloats];
     __shared__ float red[2];
 
     const int tid = threadIdx.x;
     const int rl = tid / T;                 // row within the CTA iteration
     const int tr = tid % T;                 // thread within the row
-    const int key = tid & 31;               // swizzle key of this thread's phase-B row
 
     // phase A pair j covers elements (j << SH) + 2 tr and the next one
     uint32_t sgn[4];
@@ -174,20 +180,20 @@ fwht_quant_kernel(const uint32_t *__restrict__ x,      // [M, K/2] fp16 pairs
             load_row(row0 + stride);
         fwht_bits<0, 7>(v);
 
-        // ---- transpose through shared memory (16-byte chunks XOR-swizzled)
-        float *rb = buf + rl * N;
+        // ---- transpose through shared memory: element e of the row goes to
+        // chunk e >> 7, offset e & 127; 2 tr < 2^SH never carries into the
+        // chunk index, so only the thread's base 2 tr is not a constant
+        float *rb = buf + rl * kRowFloats;
 #pragma unroll
         for (int j = 0; j < 64; ++j) {
-            const int e = (j << SH) + 2 * tr;
-            const int u = e >> 7, c = (e >> 2) & 31, wd = e & 3;
-            const int ukey = (rl * T + u) & 31;
-            *reinterpret_cast<float2 *>(rb + u * 128 + ((c ^ ukey) << 2) + wd) =
+            const int e0 = j << SH;
+            *reinterpret_cast<float2 *>(rb + 2 * tr + (e0 >> 7) * kChunk + (e0 & 127)) =
                 make_float2(v[2 * j], v[2 * j + 1]);
         }
         __syncthreads();
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-            const float4 f = *reinterpret_cast<const float4 *>(rb + tr * 128 + ((i ^ key) << 2));
+            const float4 f = *reinterpret_cast<const float4 *>(rb + tr * kChunk + 4 * i);
             v[4 * i] = f.x;
             v[4 * i + 1] = f.y;
             v[4 * i + 2] = f.z;
