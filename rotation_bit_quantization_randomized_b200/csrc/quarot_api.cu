@@ -7,6 +7,7 @@
 #include "int4_gemm.cuh"
 #include "int4_gemm_pair.cuh"
 #include "int8_gemm_pair.cuh"
+#include "kv_quant.cuh"
 #include "kv_scores.cuh"
 #include "rotate_quant.cuh"
 
@@ -531,6 +532,47 @@ quarot_status_t noalloc_scratch_address(int dev, void *&addr)
 
 }  // namespace
 
+// Tensor map of an fp16 [rows, 128] matrix (KV rows of one head) read in
+// boxes of 64 columns x 128 rows with the 128-byte swizzle.
+quarot_status_t kv_map(CUtensorMap &map, const void *base, int64_t rows)
+{
+    EncodeTiledFn fn;
+    quarot_status_t s = encode_tiled_fn(fn);
+    if (s != QUAROT_OK)
+        return s;
+    const cuuint64_t dims[2] = {128, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {256};
+    const cuuint32_t box[2] = {64, (cuuint32_t)kKvTileRows};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(QUAROT_ERR_CUDA, "cuTensorMapEncodeTiled failed (code " + std::to_string((int)r) + ")");
+    return QUAROT_OK;
+}
+
+// The staged KV-write kernel over `rows` rows of 128 elements (Hkv divides 128).
+template <bool ROTATE>
+quarot_status_t launch_kv_tma(const void *x, int64_t rows, int hkv, const int8_t *signs, uint8_t *q, void *scales,
+                              float scale_mul, float sqrt_n, cudaStream_t st, int dev, int sms)
+{
+    auto kern = kv_quant_tma_kernel<ROTATE>;
+    int per_sm = 0;
+    quarot_status_t s = kernel_occupancy(kern, dev, kKvTileRows, kKvSmemBytes, per_sm);
+    if (s != QUAROT_OK)
+        return s;
+    CUtensorMap map;
+    s = kv_map(map, x, rows);
+    if (s != QUAROT_OK)
+        return s;
+    const int64_t tiles = (rows + kKvTileRows - 1) / kKvTileRows;
+    const int grid = (int)std::min<int64_t>(tiles, (int64_t)sms * per_sm);
+    kern<<<grid, kKvTileRows, kKvSmemBytes, st>>>(map, rows, hkv, signs, q, static_cast<__half *>(scales), scale_mul,
+                                                 sqrt_n);
+    return after_launch("kv_quant_tma_kernel launch");
+}
+
 // ======================================================================= C ABI
 extern "C" {
 
@@ -731,8 +773,18 @@ quarot_status_t quarot_kv_quant(const void *k_f16, const void *v_f16, int64_t B,
         return s;
     const int64_t W = Hkv * D;
     cudaStream_t st = (cudaStream_t)stream;
-    s = launch_block<true, 128>(k_f16, rows, W, signs, kq, ks_f16, (float)(1.0 / (7.0 * std::sqrt(128.0))),
-                                (float)std::sqrt(128.0), st, dev, info->sm_count);
+    const float kmul = (float)(1.0 / (7.0 * std::sqrt(128.0)));
+    const float ksq = (float)std::sqrt(128.0);
+    if (128 % Hkv == 0 && rows * Hkv < (int64_t(1) << 31) - kKvTileRows) {
+        // rows of one head staged by the copy engine; every thread keeps one head
+        const int64_t n = rows * Hkv;
+        s = launch_kv_tma<true>(k_f16, n, (int)Hkv, signs, kq, ks_f16, kmul, ksq, st, dev, info->sm_count);
+        if (s != QUAROT_OK)
+            return s;
+        return launch_kv_tma<false>(v_f16, n, (int)Hkv, nullptr, vq, vs_f16, (float)(1.0 / 7.0), 1.0f, st, dev,
+                                    info->sm_count);
+    }
+    s = launch_block<true, 128>(k_f16, rows, W, signs, kq, ks_f16, kmul, ksq, st, dev, info->sm_count);
     if (s != QUAROT_OK)
         return s;
     return launch_block<false, 128>(v_f16, rows, W, nullptr, vq, vs_f16, (float)(1.0 / 7.0), 1.0f, st, dev,

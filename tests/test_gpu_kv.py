@@ -44,7 +44,7 @@ def _kv_check(q, k, v, s, rows=None):
     check_codes(vq, vs, oracle.f16_to_f64(vf), D)
 
 
-@pytest.mark.parametrize("B,T,H", [(1, 5, 8), (2, 64, 8), (3, 33, 1), (1, 17, 40)])
+@pytest.mark.parametrize("B,T,H", [(1, 5, 8), (2, 64, 8), (3, 33, 1), (1, 17, 40), (3, 2001, 8), (1, 700, 16)])
 def test_kv_quant_matches_oracle(q, B, T, H):
     rng = np.random.default_rng(B * 100 + T + H)
     k = (rng.standard_normal((B, T, H, 128)) * 2).astype(np.float16)
