@@ -154,15 +154,16 @@ quarot_status_t launch_fwht(const void *x, int64_t M, const int8_t *signs, uint8
                             cudaStream_t st, int dev, int sms)
 {
     auto kern = fwht_quant_kernel<LOGN, GROUP, BITS>;
+    constexpr int smem = FwhtSmem<LOGN>::kBytes;
     int per_sm = 0;
-    quarot_status_t s = kernel_occupancy(kern, dev, kFwhtThreads, 0, per_sm);
+    quarot_status_t s = kernel_occupancy(kern, dev, kFwhtThreads, smem, per_sm);
     if (s != QUAROT_OK)
         return s;
     constexpr int R = kFwhtThreads / ((1 << LOGN) / 128);
     const int64_t ctas = (M + R - 1) / R;
     const int grid = (int)std::min<int64_t>(ctas, (int64_t)sms * per_sm);
     const double n = double(1 << LOGN);
-    kern<<<grid, kFwhtThreads, 0, st>>>(reinterpret_cast<const uint32_t *>(x), M, signs, q, scales,
+    kern<<<grid, kFwhtThreads, smem, st>>>(reinterpret_cast<const uint32_t *>(x), M, signs, q, scales,
                                         (float)(1.0 / (qmax_of(BITS) * std::sqrt(n))), (float)std::sqrt(n));
     return after_launch("fwht_quant_kernel launch");
 }

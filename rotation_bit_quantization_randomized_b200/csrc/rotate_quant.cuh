@@ -35,6 +35,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "tc_ptx.cuh"
 
 namespace quarot {
 
@@ -114,6 +115,30 @@ __device__ __forceinline__ float group_scale(float amax, float scale_mul, float 
 // ---------------------------------------------------------------------------
 // Full transform, K = 2^LOGN with 8 <= LOGN <= 13.
 // ---------------------------------------------------------------------------
+
+// Shared-memory plan of fwht_quant_kernel (dynamic shared memory).
+template <int LOGN>
+struct FwhtSmem {
+    static constexpr int N = 1 << LOGN;
+    static constexpr int T = N / 128;                   // threads per row
+    static constexpr int R = kFwhtThreads / T;          // rows per CTA iteration
+    // staging: one slot per row, padded so that the phase-A reads of a warp
+    // spanning several rows fall on different banks
+    static constexpr int kPadWords = (T >= 32 || T < 4) ? 4 : T;
+    static constexpr int kStageRowBytes = N * 2 + 4 * kPadWords;
+    static constexpr int kStageBytes = R * kStageRowBytes;
+    // transpose buffer: each 128-element chunk padded to 132 floats and each
+    // row by 4 more (8 at K = 1024), so that the phase-A writes of a warp take
+    // 2 wavefronts per 256 B and its phase-B reads 4 per 512 B (the minimum)
+    // at every K, and every address is a per-thread base plus a constant
+    static constexpr int kChunk = 132;
+    static constexpr int kRowFloats = (N / 128) * kChunk + (LOGN == 10 ? 8 : 4);
+    static constexpr int kBufOffset = kStageBytes;
+    static constexpr int kBarOffset = kBufOffset + R * kRowFloats * 4;
+    static constexpr int kBytes = kBarOffset + 16 + 16;
+    static_assert(kStageRowBytes % 16 == 0 && kBufOffset % 16 == 0, "16-byte aligned staging and buffer");
+};
+
 template <int LOGN, int GROUP, int BITS = 4>
 __global__ void __launch_bounds__(kFwhtThreads, 4)
 fwht_quant_kernel(const uint32_t *__restrict__ x,      // [M, K/2] fp16 pairs
@@ -125,22 +150,20 @@ fwht_quant_kernel(const uint32_t *__restrict__ x,      // [M, K/2] fp16 pairs
 {
     static_assert(LOGN >= 8 && LOGN <= 13, "full transform covers 256..8192");
     static_assert(BITS == 4 || (BITS == 8 && GROUP == 0), "8-bit codes use one scale per row");
+    using S = FwhtSmem<LOGN>;
     constexpr float kQmax = BITS == 8 ? 127.0f : 7.0f;
-    constexpr int N = 1 << LOGN;
-    constexpr int T = N / 128;              // threads per row
-    constexpr int R = kFwhtThreads / T;     // rows per CTA iteration
+    constexpr int N = S::N;
+    constexpr int T = S::T;
+    constexpr int R = S::R;
     constexpr int SH = LOGN - 6;            // element shift of the phase-A pair index j
     constexpr int PB = (LOGN - 7) < 6 ? (LOGN - 7) : 6;   // phase-B bits 1..PB
+    constexpr int kChunk = S::kChunk;
+    constexpr int kRowFloats = S::kRowFloats;
 
-    // transpose buffer: each 128-element chunk padded to 132 floats and each
-    // row of the CTA iteration by 4 more (8 at K = 1024), so that the phase-A
-    // writes of a warp take 2 wavefronts per 256 B and its phase-B reads 4 per
-    // 512 B (the minimum) at every K, and every address is a per-thread base
-    // plus a compile-time offset
-    constexpr int kChunk = 132;
-    constexpr int kRowFloats = (N / 128) * kChunk + (LOGN == 10 ? 8 : 4);
-    __shared__ __align__(16) float buf[R * kRowFloats];
-    __shared__ float red[2];
+    extern __shared__ __align__(128) uint8_t fwht_smem[];
+    float *buf = reinterpret_cast<float *>(fwht_smem + S::kBufOffset);
+    const uint32_t bar = smem_u32(fwht_smem + S::kBarOffset);
+    float *red = reinterpret_cast<float *>(fwht_smem + S::kBarOffset + 16);
 
     const int tid = threadIdx.x;
     const int rl = tid / T;                 // row within the CTA iteration
@@ -150,34 +173,54 @@ fwht_quant_kernel(const uint32_t *__restrict__ x,      // [M, K/2] fp16 pairs
     uint32_t sgn[4];
     build_sign_words(signs, [&](int j) { return (j << SH) + 2 * tr; }, sgn);
 
-    // raw fp16 pairs of the next row this thread handles: loaded one row ahead
-    // so that the loads overlap the transform of the current row
-    uint32_t nxt[64];
-    auto load_row = [&](int64_t r0) {
-        const int64_t r = r0 + rl;
-        const bool ok = r < M;
-        const uint32_t *xr = x + (ok ? r : 0) * (N / 2);
-#pragma unroll
-        for (int j = 0; j < 64; ++j)
-            nxt[j] = ok ? __ldg(xr + (j << (SH - 1)) + tr) : 0u;
-    };
+    // The fp16 rows of the next iteration are copied by the bulk copy engine
+    // into the staging slots while this iteration finishes (issued once every
+    // thread has read the slots), so no register holds data in flight.
     const int64_t stride = (int64_t)gridDim.x * R;
-    load_row((int64_t)blockIdx.x * R);
+    auto issue = [&](int64_t r0) {
+        const int nrows = (int)min((int64_t)R, M - r0);
+        mbar_arrive_expect_tx(bar, (uint32_t)(nrows * N * 2));
+        for (int rr = 0; rr < nrows; ++rr)
+            bulk_load(smem_u32(fwht_smem + rr * S::kStageRowBytes), x + (r0 + rr) * (N / 2), N * 2, bar);
+    };
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        mbar_fence_init();
+    }
+    __syncthreads();
+    if (tid == 0 && (int64_t)blockIdx.x * R < M)
+        issue((int64_t)blockIdx.x * R);
 
-    for (int64_t row0 = (int64_t)blockIdx.x * R; row0 < M; row0 += stride) {
+    const uint32_t *stage = reinterpret_cast<const uint32_t *>(fwht_smem + rl * S::kStageRowBytes);
+    int it = 0;
+    bool ok = true;
+    for (int64_t row0 = (int64_t)blockIdx.x * R; row0 < M; row0 += stride, ++it) {
         const int64_t row = row0 + rl;
         const bool valid = row < M;
 
+        if (!mbar_try_wait(bar, (uint32_t)it & 1)) {
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(bar, (uint32_t)it & 1)) {
+                if (globaltimer_ns() - t0 > 2000000000ull) {
+                    record_timeout();
+                    ok = false;
+                    break;
+                }
+            }
+        }
+        if (!__syncthreads_and(ok))
+            break;
+
         // ---- phase A: register r = 2 j + b holds element (j << SH) + 2 tr + b
+        // (rows past M were not copied: their slots hold stale data, and
+        // nothing computed from them is stored)
         float v[128];
 #pragma unroll
         for (int j = 0; j < 64; ++j) {
-            const float2 f = half2_bits_to_float2(apply_sign_pair(nxt[j], sgn, j));
+            const float2 f = half2_bits_to_float2(apply_sign_pair(stage[(j << (SH - 1)) + tr], sgn, j));
             v[2 * j] = f.x;
             v[2 * j + 1] = f.y;
         }
-        if (row0 + stride < M)
-            load_row(row0 + stride);
         fwht_bits<0, 7>(v);
 
         // ---- transpose through shared memory: element e of the row goes to
@@ -191,6 +234,9 @@ fwht_quant_kernel(const uint32_t *__restrict__ x,      // [M, K/2] fp16 pairs
                 make_float2(v[2 * j], v[2 * j + 1]);
         }
         __syncthreads();
+        // every thread has read its staging slot: refill it for the next iteration
+        if (tid == 0 && row0 + stride < M)
+            issue(row0 + stride);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             const float4 f = *reinterpret_cast<const float4 *>(rb + tr * kChunk + 4 * i);
@@ -234,6 +280,12 @@ fwht_quant_kernel(const uint32_t *__restrict__ x,      // [M, K/2] fp16 pairs
             quant_store_i8(v, r, reinterpret_cast<int8_t *>(q) + (valid ? row : 0) * N + tr * 128, valid);
         else
             quant_pack_store<GROUP>(v, r, q + (valid ? row : 0) * (N / 2) + tr * 64, valid);
+    }
+    // after an abort, a copy may still be in flight into this CTA's memory
+    if (!ok && tid == 0) {
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 1000000ull) {
+        }
     }
     // a dependent GEMM launched with programmatic serialization may start now
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
