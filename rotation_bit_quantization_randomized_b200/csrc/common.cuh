@@ -135,6 +135,24 @@ __device__ __forceinline__ void fma_x2(float a0, float a1, float b, float c, flo
         : "f"(a0), "f"(a1), "f"(b), "f"(c));
 }
 
+// (d0, d1) = (a0 - c, a1 - c) with one packed fp32x2 subtract.
+__device__ __forceinline__ void sub_x2(float a0, float a1, float c, float &d0, float &d1)
+{
+    asm("{\n\t.reg .b64 ra, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rc, {%4, %4};\n\t"
+        "sub.rn.f32x2 rd, ra, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(c));
+}
+
+// (acc0, acc1) += (a0 * b, a1 * b) with one packed fp32x2 fused multiply-add.
+__device__ __forceinline__ void fma_x2_acc(float a0, float a1, float b, float &acc0, float &acc1)
+{
+    asm("{\n\t.reg .b64 ra, rb, rc;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\t"
+        "mov.b64 rc, {%0, %1};\n\tfma.rn.f32x2 rc, ra, rb, rc;\n\tmov.b64 {%0, %1}, rc;\n\t}"
+        : "+f"(acc0), "+f"(acc1)
+        : "f"(a0), "f"(a1), "f"(b));
+}
+
 __device__ __forceinline__ float warp_max(float v, int width)
 {
 #pragma unroll

@@ -37,22 +37,56 @@ kv_scores_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
     const int Hq = Hkv * G;
     const int tid = threadIdx.x;
 
-    // rotate the G queries of this kv-head: thread g < G owns head g
-    if (tid < G) {
-        const __half2 *qh = reinterpret_cast<const __half2 *>(q + (b * Hq + (int64_t)h * G + tid) * 128);
-        const int8_t *sg = signs + h * 128;
-        float v[128];
+    // rotate the G queries of this kv-head cooperatively: 16 threads per
+    // query (a half warp), thread p of a query holding elements 8p .. 8p+7;
+    // the Walsh-Hadamard stages on element bits 0-2 run in registers, those
+    // on bits 3-6 (= bits of p) through half-warp shuffles
+    {
+        const int p = tid & 15;
+        const int8_t *sg = signs + h * 128 + 8 * p;
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-            float2 f = __half22float2(qh[j]);
-            v[2 * j] = sg[2 * j] < 0 ? -f.x : f.x;
-            v[2 * j + 1] = sg[2 * j + 1] < 0 ? -f.y : f.y;
+        for (int g0 = 0; g0 < G; g0 += kScoreThreads / 16) {
+            // every lane runs the shuffles; lanes of a query index >= G only
+            // skip their load and store
+            const int g = g0 + (tid >> 4);
+            const bool gv = G % (kScoreThreads / 16) == 0 || g < G;
+            {
+                const uint4 raw = gv ? *reinterpret_cast<const uint4 *>(q + (b * Hq + (int64_t)h * G + g) * 128 + 8 * p)
+                                     : make_uint4(0u, 0u, 0u, 0u);
+                const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+                float v[8];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float2 f = half2_bits_to_float2(w4[k]);
+                    v[2 * k] = sg[2 * k] < 0 ? -f.x : f.x;
+                    v[2 * k + 1] = sg[2 * k + 1] < 0 ? -f.y : f.y;
+                }
+#pragma unroll
+                for (int hb = 1; hb < 8; hb <<= 1)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        if ((i & hb) == 0) {
+                            const float a = v[i], c = v[i + hb];
+                            v[i] = a + c;
+                            v[i + hb] = a - c;
+                        }
+#pragma unroll
+                for (int lb = 1; lb < 16; lb <<= 1) {
+                    const bool upper = (p & lb) != 0;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float o = __shfl_xor_sync(0xffffffffu, v[i], lb);
+                        v[i] = upper ? o - v[i] : v[i] + o;
+                    }
+                }
+                const float inv = 0.08838834764831845f;   // 1/sqrt(128)
+                if (gv) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        qs[8 * p + i][g] = v[i] * inv;
+                }
+            }
         }
-        fwht_bits<0, 7>(v);
-        const float inv = 0.08838834764831845f;       // 1/sqrt(128)
-#pragma unroll
-        for (int d = 0; d < 128; ++d)
-            qs[d][tid] = v[d] * inv;
     }
     __syncthreads();
 
@@ -85,29 +119,31 @@ kv_scores_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
 #pragma unroll
         for (int wd = 0; wd < 4; ++wd) {
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
+            for (int k = 0; k < 8; k += 2) {
                 const int d = qd * 32 + wd * 8 + k;
-                float qv[G];
+                float qv0[G], qv1[G];                 // queries at d and d + 1
 #pragma unroll
-                for (int g = 0; g < G; g += 4) {
-                    if (G >= 4) {
-                        const float4 f = *reinterpret_cast<const float4 *>(&qs[d][g]);
-                        qv[g] = f.x; qv[g + 1] = f.y; qv[g + 2] = f.z; qv[g + 3] = f.w;
-                    } else {
-#pragma unroll
-                        for (int gg = 0; gg < G; ++gg)
-                            qv[gg] = qs[d][gg];
-                    }
+                for (int g = 0; g < G; ++g) {
+                    qv0[g] = qs[d][g];
+                    qv1[g] = qs[d + 1][g];
                 }
 #pragma unroll
                 for (int i = 0; i < kScoreTokPerThread; ++i) {
                     const uint32_t word = wd == 0 ? cur[i].x : wd == 1 ? cur[i].y : wd == 2 ? cur[i].z : cur[i].w;
-                    // nibble -> float exactly: (2^23 + (c ^ 8)) - (2^23 + 8) = c
-                    const uint32_t u = ((word >> (4 * k)) & 0xFu) ^ 0x4B000008u;
-                    const float c = __uint_as_float(u) - 8388616.0f;
+                    // two nibbles -> two floats exactly with one packed subtract:
+                    // (2^23 + (c ^ 8)) - (2^23 + 8) = c
+                    float c0, c1;
+                    sub_x2(__uint_as_float(((word >> (4 * k)) & 0xFu) ^ 0x4B000008u),
+                           __uint_as_float(((word >> (4 * k + 4)) & 0xFu) ^ 0x4B000008u), 8388616.0f, c0, c1);
 #pragma unroll
-                    for (int g = 0; g < G; ++g)
-                        acc[i][g] = fmaf(qv[g], c, acc[i][g]);
+                    for (int g = 0; g + 1 < G; g += 2) {
+                        fma_x2_acc(qv0[g], qv0[g + 1], c0, acc[i][g], acc[i][g + 1]);
+                        fma_x2_acc(qv1[g], qv1[g + 1], c1, acc[i][g], acc[i][g + 1]);
+                    }
+                    if (G & 1) {
+                        acc[i][G - 1] = fmaf(qv0[G - 1], c0, acc[i][G - 1]);
+                        acc[i][G - 1] = fmaf(qv1[G - 1], c1, acc[i][G - 1]);
+                    }
                 }
             }
         }
