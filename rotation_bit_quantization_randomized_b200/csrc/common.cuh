@@ -144,6 +144,15 @@ __device__ __forceinline__ void sub_x2(float a0, float a1, float c, float &d0, f
         : "f"(a0), "f"(a1), "f"(c));
 }
 
+// (d0, d1) = (a0 * b0, a1 * b1) with one packed fp32x2 multiply.
+__device__ __forceinline__ void mul_x2(float a0, float a1, float b0, float b1, float &d0, float &d1)
+{
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // (acc0, acc1) += (a0 * b, a1 * b) with one packed fp32x2 fused multiply-add.
 __device__ __forceinline__ void fma_x2_acc(float a0, float a1, float b, float &acc0, float &acc1)
 {

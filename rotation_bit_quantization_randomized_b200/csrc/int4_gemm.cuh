@@ -73,13 +73,15 @@ struct GemmShape {
     static constexpr int kTmaWarp = kEpiWarps + 1;
     static constexpr int kUnpackWarp0 = kEpiWarps + 2;
     static constexpr int kThreads = 32 * (kUnpackWarp0 + kUnpackWarps);
-    static constexpr int kTmemCols = 2 * BN;
+    // two accumulators in tensor memory (the grouped epilogue uses one per K block)
+    static constexpr int kAccBufs = 2;
+    static constexpr int kTmemCols = kAccBufs * BN;
     static constexpr int kIntOffset = kPStages * kPackedStage;  // int8 ring after the packed ring
     static constexpr int kBarOffset = kIntOffset + kIStages * kStageBytes;
-    static constexpr int kNumBars = 2 * kPStages + 2 * kIStages + 7;
+    static constexpr int kNumBars = 2 * kPStages + 2 * kIStages + 2 * kAccBufs + 1;
     static constexpr int kMiscOffset = kBarOffset + 8 * kNumBars;
     static constexpr int kSwOffset = kMiscOffset + 16;
-    static constexpr int kSmemBytes = kSwOffset + 2 * BN * 4 + 1024;
+    static constexpr int kSmemBytes = kSwOffset + 2 * 8 * (kGemmBM + BN) * 4 + 1024;   // grouped scale chunks
     static_assert(kStageBytes % 1024 == 0 && kIntOffset % 1024 == 0, "int8 stages keep 1024-byte alignment");
     static_assert(kPackedStage % 1024 == 0, "packed stages keep 1024-byte alignment");
     static_assert(kGemmBM % (8 * kGroupsPerWarp) == 0, "an unpack warp handles only A or only B rows");
@@ -152,13 +154,21 @@ __device__ __forceinline__ bool gemm_wait_drain(uint32_t bar, uint32_t parity)
     return true;
 }
 
-__device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
-
-// int32 with |v| < 2^22 to float exactly, without the slow conversion unit.
-__device__ __forceinline__ float small_i2f(uint32_t v)
+// Named barrier 1 among the first `nthreads` threads (the epilogue warps)
+// that also returns the AND of every participant's `p`.
+__device__ __forceinline__ bool epi_barrier_and(int nthreads, bool p)
 {
-    return __uint_as_float(v + 0x4B400000u) - 12582912.0f;
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.and.pred po, 1, %2, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)p), "r"(nthreads)
+        : "memory");
+    return r != 0;
 }
+
+__device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
 
 template <int BN, int EPI>
 __global__ void __launch_bounds__(GemmShape<BN, EPI>::kThreads, 1)
@@ -174,9 +184,8 @@ int4_gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_a,
     const uint32_t bar_ifull = bar_pempty + 8 * S::kPStages;
     const uint32_t bar_iempty = bar_ifull + 8 * S::kIStages;
     const uint32_t bar_accf = bar_iempty + 8 * S::kIStages;
-    const uint32_t bar_acce = bar_accf + 16;
-    const uint32_t bar_drain = bar_acce + 16;
-    const uint32_t bar_sws = bar_drain + 8;        // grouped: column-scale staging, 2 buffers
+    const uint32_t bar_acce = bar_accf + 8 * S::kAccBufs;
+    const uint32_t bar_drain = bar_acce + 8 * S::kAccBufs;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + S::kMiscOffset);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + S::kMiscOffset + 4);
 
@@ -196,13 +205,11 @@ int4_gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_a,
             mbar_init(bar_ifull + 8 * s, S::kUnpackThreads);
             mbar_init(bar_iempty + 8 * s, 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < S::kAccBufs; ++b) {
             mbar_init(bar_accf + 8 * b, 1);
             mbar_init(bar_acce + 8 * b, S::kEpiThreads);
         }
         mbar_init(bar_drain, 1);
-        mbar_init(bar_sws, S::kEpiThreads);
-        mbar_init(bar_sws + 8, S::kEpiThreads);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -309,8 +316,8 @@ int4_gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_a,
             int step = 0;
             for (int lt = 0; lt < my_tiles && ok; ++lt) {
                 for (int kb = 0; kb < KB && ok; ++kb, ++step) {
-                    const int ab = EPI == kEpiGroupF16 ? (step & 1) : (lt & 1);
-                    const uint32_t ause = EPI == kEpiGroupF16 ? (uint32_t)(step >> 1) : (uint32_t)(lt >> 1);
+                    const int ab = EPI == kEpiGroupF16 ? (step % S::kAccBufs) : (lt & 1);
+                    const uint32_t ause = EPI == kEpiGroupF16 ? (uint32_t)(step / S::kAccBufs) : (uint32_t)(lt >> 1);
                     if (EPI == kEpiGroupF16 || kb == 0) {
                         if (!gemm_wait(bar_acce + 8 * ab, (ause & 1) ^ 1, abort_flag)) {
                             ok = false;
@@ -407,47 +414,108 @@ int4_gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_a,
                     }
                 }
             } else {
-                // grouped: warps w and w+4 share TMEM lanes and split the columns
+                // grouped: warps w and w+4 share TMEM lanes and split the columns.
+                // The scales of 8 K groups at a time are staged in shared memory
+                // one chunk ahead (threads 0-127 the tile's row scales, 128-255
+                // its column scales), so no step waits on a global load; a
+                // named barrier of the epilogue warps hands each chunk over.
                 constexpr int HALF = BN / 2;
+                constexpr int kCh = 8;                           // K groups per staged chunk
+                static_assert(S::kEpiThreads == kGemmBM + BN, "one staging thread per tile row and column");
                 const int col0 = (warp >> 2) * HALF;
                 const int et = threadIdx.x;                      // 0 .. kEpiThreads-1
                 const int G = KB;
+                float *sac = reinterpret_cast<float *>(smem + S::kSwOffset);       // [2][kCh][kGemmBM]
+                float *swc = sac + 2 * kCh * kGemmBM;                              // [2][kCh][BN]
+                const bool is_row = et < kGemmBM;
+                const int64_t srow = is_row ? (int64_t)mb * kGemmBM + et : n0 + (et - kGemmBM);
+                const bool sval = is_row ? srow < a.M : srow < a.N;
+                const __half *sptr = reinterpret_cast<const __half *>(is_row ? a.sa : a.sw) + (sval ? srow : 0) * G;
+                const float smul = is_row ? (1.0f / 256.0f) : 1.0f;
+                auto load_chunk = [&](int kb0, float (&d)[kCh]) {
+                    if (sval && G % kCh == 0) {
+                        const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(sptr + kb0));
+                        const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float2 f = half2_bits_to_float2(w4[i]);
+                            d[2 * i] = f.x * smul;
+                            d[2 * i + 1] = f.y * smul;
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < kCh; ++i)
+                            d[i] = (sval && kb0 + i < G) ? __half2float(sptr[kb0 + i]) * smul : 0.f;
+                    }
+                };
+                auto store_chunk = [&](int cb, const float (&d)[kCh]) {
+#pragma unroll
+                    for (int i = 0; i < kCh; ++i) {
+                        if (is_row)
+                            sac[(cb * kCh + i) * kGemmBM + et] = d[i];
+                        else
+                            swc[(cb * kCh + i) * BN + (et - kGemmBM)] = d[i];
+                    }
+                };
                 float accv[HALF];
 #pragma unroll
                 for (int i = 0; i < HALF; ++i)
                     accv[i] = 0.f;
-                for (int kb = 0; kb < KB; ++kb, ++step) {
-                    const int ab = step & 1;
-                    float *sws = reinterpret_cast<float *>(smem + S::kSwOffset) + ab * BN;
-                    if (et < BN) {
-                        const int64_t n = n0 + et;
-                        sws[et] = n < a.N ? __half2float(reinterpret_cast<const __half *>(a.sw)[n * G + kb]) : 0.f;
-                    }
-                    mbar_arrive(bar_sws + 8 * ab);
-                    if (!gemm_wait(bar_sws + 8 * ab, (uint32_t)(step >> 1) & 1, abort_flag) ||
-                        !gemm_wait(bar_accf + 8 * ab, (uint32_t)(step >> 1) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const float sag = mrow ? __half2float(reinterpret_cast<const __half *>(a.sa)[m * G + kb]) *
-                                                 (1.0f / 256.0f)
-                                           : 0.f;
-#pragma unroll
-                    for (int c = 0; c < HALF / 16; ++c) {
-                        uint32_t r[16];
-                        __syncwarp();
-                        tmem_ld16(lane_addr + ab * BN + col0 + 16 * c, r);
-                        tmem_wait_ld16(r);
-                        if (c == HALF / 16 - 1) {
-                            tc_fence_before();
-                            mbar_arrive(bar_acce + 8 * ab);
-                        }
-#pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            accv[16 * c + i] = fmaf(small_i2f(r[i]) * sag, sws[col0 + 16 * c + i], accv[16 * c + i]);
-                    }
+                {
+                    float d[kCh];
+                    load_chunk(0, d);
+                    store_chunk(0, d);
                 }
+                for (int kb0 = 0; kb0 < KB; kb0 += kCh) {
+                    const int cb = (kb0 / kCh) & 1;
+                    // chunk cb is complete, and nobody still reads chunk cb ^ 1;
+                    // the barrier also makes every epilogue thread's decision to
+                    // go on (or to give up after a timeout) the same
+                    ok = epi_barrier_and(S::kEpiThreads, ok);
+                    if (!ok)
+                        break;
+                    float nxt[kCh];
+                    if (kb0 + kCh < KB)
+                        load_chunk(kb0 + kCh, nxt);
+                    const int nu = min(kCh, KB - kb0);
+                    for (int u = 0; u < nu; ++u, ++step) {
+                        const int ab = step % S::kAccBufs;
+                        const uint32_t par = (uint32_t)(step / S::kAccBufs) & 1;
+                        if (!gemm_wait(bar_accf + 8 * ab, par, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const float sag = sac[(cb * kCh + u) * kGemmBM + 32 * wq + lane];
+                        const float *sws = swc + (cb * kCh + u) * BN;
+#pragma unroll
+                        for (int c = 0; c < HALF / 16; ++c) {
+                            uint32_t r[16];
+                            __syncwarp();
+                            tmem_ld16(lane_addr + ab * BN + col0 + 16 * c, r);
+                            tmem_wait_ld16(r);
+                            if (c == HALF / 16 - 1) {
+                                tc_fence_before();
+                                mbar_arrive(bar_acce + 8 * ab);
+                            }
+                            // two partial sums at a time: exact int -> float with one
+                            // packed subtract (|acc| < 2^22), times the column scales,
+                            // then accumulated with the row scale by one packed FMA
+#pragma unroll
+                            for (int i = 0; i < 16; i += 2) {
+                                float f0, f1;
+                                sub_x2(__uint_as_float(r[i] + 0x4B400000u), __uint_as_float(r[i + 1] + 0x4B400000u),
+                                       12582912.0f, f0, f1);
+                                const float2 w = *reinterpret_cast<const float2 *>(sws + col0 + 16 * c + i);
+                                mul_x2(f0, f1, w.x, w.y, f0, f1);
+                                fma_x2_acc(f0, f1, sag, accv[16 * c + i], accv[16 * c + i + 1]);
+                            }
+                        }
+                    }
+                    if (kb0 + kCh < KB)
+                        store_chunk(cb ^ 1, nxt);
+                }
+                ok = epi_barrier_and(S::kEpiThreads, ok);
                 if (!ok)
                     break;
                 if (mrow) {
