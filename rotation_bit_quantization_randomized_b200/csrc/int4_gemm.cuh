@@ -73,8 +73,9 @@ struct GemmShape {
     static constexpr int kTmaWarp = kEpiWarps + 1;
     static constexpr int kUnpackWarp0 = kEpiWarps + 2;
     static constexpr int kThreads = 32 * (kUnpackWarp0 + kUnpackWarps);
-    // two accumulators in tensor memory (the grouped epilogue uses one per K block)
-    static constexpr int kAccBufs = 2;
+    // accumulators in tensor memory: two per-tile buffers, or (grouped) four
+    // per-K-block buffers so that the MMA runs ahead of the rescale
+    static constexpr int kAccBufs = EPI == kEpiGroupF16 ? 4 : 2;
     static constexpr int kTmemCols = kAccBufs * BN;
     static constexpr int kIntOffset = kPStages * kPackedStage;  // int8 ring after the packed ring
     static constexpr int kBarOffset = kIntOffset + kIStages * kStageBytes;
