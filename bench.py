@@ -62,24 +62,36 @@ def peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, src="of fallback")
 
 
-def source_hash():
+# device-source files each profiled kernel is compiled from
+KERNEL_SOURCES = {
+    "int4_gemm_pair_kernel": ["int4_gemm_pair.cuh", "int4_gemm.cuh", "tc_ptx.cuh", "common.cuh"],
+    "fwht_quant_kernel": ["rotate_quant.cuh", "tc_ptx.cuh", "common.cuh"],
+    "kv_quant_tma_kernel_keys": ["kv_quant.cuh", "rotate_quant.cuh", "tc_ptx.cuh", "common.cuh"],
+    "kv_scores_kernel": ["kv_scores.cuh", "common.cuh"],
+}
+
+
+def source_hash(kernel=None):
+    """Hash of the library sources (all of csrc/), or of one kernel's device sources."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "rotation_bit_quantization_randomized_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    files = sorted(os.listdir(csrc)) if kernel is None else KERNEL_SOURCES[kernel]
+    for f in files:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel):
-    """DRAM bytes per launch from the committed ncu summary, if taken on this source."""
+    """DRAM bytes per launch from the committed ncu summary, if taken on the
+    kernel's current device sources (null once the kernel has changed)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
     e = d.get(kernel)
-    if not e or e.get("source_sha") != source_hash():
+    if not e or kernel not in KERNEL_SOURCES or e.get("source_sha") != source_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -362,11 +374,11 @@ def run_ours(args, rank, world, local_rank, dist):
             "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N, "kv": [c.B, c.T, c.Hkv, c.D], "q_heads": c.Hq,
                        "l2": "inputs and outputs larger than L2; no explicit flush",
                        "parallelism": f"replicas x{world}"},
-            "roofline": {"bound": "tensor", "kernel": "int4_gemm_pair_kernel<0> (quarot_int4_linear)",
+            "roofline": {"bound": "tensor", "kernel": "int4_gemm_pair_kernel<224,0> (quarot_int4_linear)",
                          "achieved": gemm_tops, "peak": int8_sust, "unit": "TFLOP/s",
                          "frac": gemm_tops / int8_sust, "traffic": traffic,
                          "peak_note": f"int8 dense = 2 x bf16 sustained {pk['bf16_sust']} {pk['src']}"},
-            "rotate_quant_roofline": {"bound": "hbm", "kernel": "fwht_quant_kernel<13,0> (quarot_rotate_quant)",
+            "rotate_quant_roofline": {"bound": "hbm", "kernel": "fwht_quant_kernel<13,0,4> (quarot_rotate_quant)",
                                       "achieved": rq_gbs, "peak": pk["hbm"], "unit": "GB/s",
                                       "frac": rq_gbs / pk["hbm"], "traffic": recorded_traffic("fwht_quant_kernel"),
                                       "peak_note": f"HBM copy {pk['src']}"},
