@@ -42,6 +42,8 @@ def lib():
             "qo_quantize": [P, I64, I64, I64, P, P, P],
             "qo_quantize_with_scales": [P, I64, I64, I64, P, P],
             "qo_quantize_bits": [P, I64, I64, ctypes.c_int, P, P],
+            "qo_quantize_asym": [P, I64, I64, ctypes.c_int, ctypes.c_double, P, P, P, P],
+            "qo_dequant_asym": [P, I64, I64, I64, P, P, P, P, P, P, P, P],
             "qo_quantize_bits_with_scales": [P, I64, I64, ctypes.c_int, P, P],
             "qo_pack": [P, I64, P],
             "qo_unpack": [P, I64, P],
@@ -198,6 +200,54 @@ def linear8(x16, w16, signs, had_block: int = 0):
     acc = int_gemm(qa, qw, 0)
     y, y16 = dequant_linear(acc, sa, sw, 0)
     return dict(qa=qa, sa=sa, qw=qw, sw=sw, acc=acc, y=y, y16=y16)
+
+
+def quantize_asym(xr, clip: float, bits: int = 4):
+    """Per-row asymmetric RTN with clipping: (codes int8 in [0, 2^bits-1] [M, K],
+    step fp64 [M], zero point int64 [M], code row sums int64 [M])."""
+    xr = _c(xr, np.float64)
+    M, K = xr.shape
+    codes = np.empty((M, K), np.int8)
+    d = np.empty((M,), np.float64)
+    z = np.empty((M,), np.int64)
+    r = np.empty((M,), np.int64)
+    _check(lib().qo_quantize_asym(_p(xr), M, K, bits, float(clip), _p(codes), _p(d), _p(z), _p(r)),
+           "quantize_asym")
+    return codes, d, z, r
+
+
+def dequant_asym(acc, K, da, za, ra, dw, zw, rw):
+    """y = da dw (acc - zw ra - za rw + K za zw).  Returns (y fp64, y fp16 bits)."""
+    acc = _c(np.asarray(acc, np.int64), np.int64)
+    M, N = acc.shape
+    y = np.empty((M, N), np.float64)
+    y16 = np.empty((M, N), np.uint16)
+    _check(lib().qo_dequant_asym(_p(acc), M, N, K, _p(_c(da, np.float64)), _p(_c(za, np.int64)),
+                                 _p(_c(ra, np.int64)), _p(_c(dw, np.float64)), _p(_c(zw, np.int64)),
+                                 _p(_c(rw, np.int64)), _p(y), _p(y16)), "dequant_asym")
+    return y, y16
+
+
+def rotate_quant_asym(x16, signs, clip: float, had_block: int = 0):
+    """Rotate, then per-row asymmetric 4-bit RTN with clipping, packed (low nibble =
+    even element).  Returns (packed, step, zero, rowsum, x')."""
+    xr = rotate(x16, signs, had_block)
+    codes, d, z, r = quantize_asym(xr, clip, 4)
+    return pack(codes), d, z, r, xr
+
+
+def linear_asym(x16, w16, signs, clip_a: float = 0.9, clip_w: float = 0.8, had_block: int = 0):
+    """The asymmetric INT4 linear: activations per token (clip_a), weights per
+    output channel (clip_w), integer product of the unsigned codes and the
+    zero-point-corrected dequantized output."""
+    qa, da, za, ra, _ = rotate_quant_asym(x16, signs, clip_a, had_block)
+    qw, dw, zw, rw, _ = rotate_quant_asym(w16, signs, clip_w, had_block)
+    ua = unpack(qa) & 0x0F
+    uw = unpack(qw) & 0x0F
+    acc = int_gemm(ua, uw, 0)
+    K = ua.shape[1]
+    y, y16 = dequant_asym(acc, K, da, za, ra, dw, zw, rw)
+    return dict(qa=qa, da=da, za=za, ra=ra, qw=qw, dw=dw, zw=zw, rw=rw, acc=acc, y=y, y16=y16)
 
 
 def pack(codes) -> np.ndarray:

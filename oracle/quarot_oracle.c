@@ -354,6 +354,86 @@ int qo_quantize_bits_with_scales(const double *xr, int64_t M, int64_t K, int bit
     return 0;
 }
 
+/* ------------------------------------------------------------------------ */
+/* Asymmetric RTN with a clipping ratio (DuQuant, Knowl 12: per-token         */
+/* asymmetric activations, per-channel asymmetric weights, clipping ratios    */
+/* 0.9 / 0.8 on the extremes; the step of its clipped range is                */
+/* (gamma max - beta min) / (2^b - 1), here gamma = beta = the ratio).        */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Per row: lo = clip * min, hi = clip * max, step d = (hi - lo) / (2^bits - 1),
+ * zero point z = rint(-lo / d), codes u = clamp(rint(v / d) + z, 0, 2^bits - 1)
+ * (ties to even), so that v is reconstructed as d * (u - z).  A zero step
+ * gives zero codes and zero point.  Outputs: codes (one per int8, values
+ * 0 .. 2^bits - 1), step (fp64), zero point and the row's code sum (int64).
+ */
+int qo_quantize_asym(const double *xr, int64_t M, int64_t K, int bits, double clip, int8_t *codes,
+                     double *step, int64_t *zero, int64_t *rowsum)
+{
+    if (M < 0 || K <= 0 || bits < 2 || bits > 8 || !(clip > 0.0) || clip > 1.0)
+        return -1;
+    const double qmax = (double)((1 << bits) - 1);
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; ++r) {
+        const double *v = xr + r * K;
+        double mn = v[0], mx = v[0];
+        for (int64_t k = 1; k < K; ++k) {
+            if (v[k] < mn)
+                mn = v[k];
+            if (v[k] > mx)
+                mx = v[k];
+        }
+        const double lo = clip * mn, hi = clip * mx;
+        const double d = (hi - lo) / qmax;
+        int64_t z = 0, sum = 0;
+        if (d > 0.0)
+            z = (int64_t)nearbyint(-lo / d);
+        for (int64_t k = 0; k < K; ++k) {
+            int64_t u = 0;
+            if (d > 0.0) {
+                double q = nearbyint(v[k] / d) + (double)z;
+                if (q < 0.0)
+                    q = 0.0;
+                if (q > qmax)
+                    q = qmax;
+                u = (int64_t)q;
+            }
+            codes[r * K + k] = (int8_t)u;
+            sum += u;
+        }
+        step[r] = d;
+        zero[r] = z;
+        rowsum[r] = sum;
+    }
+    return 0;
+}
+
+/*
+ * The dequantized product of asymmetric codes:
+ *   y[m, n] = da[m] dw[n] sum_k (ua[m,k] - za[m]) (uw[n,k] - zw[n])
+ *           = da[m] dw[n] (acc[m,n] - zw[n] ra[m] - za[m] rw[n] + K za[m] zw[n])
+ * with acc = sum_k ua uw (int64) and ra, rw the row code sums; the integer
+ * bracket is formed exactly, then scaled in fp64.
+ */
+int qo_dequant_asym(const int64_t *acc, int64_t M, int64_t N, int64_t K, const double *da, const int64_t *za,
+                    const int64_t *ra, const double *dw, const int64_t *zw, const int64_t *rw, double *y64,
+                    uint16_t *y16)
+{
+    if (M < 0 || N < 0 || K <= 0)
+        return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            const int64_t b = acc[m * N + n] - zw[n] * ra[m] - za[m] * rw[n] + K * za[m] * zw[n];
+            const double y = (double)b * da[m] * dw[n];
+            y64[m * N + n] = y;
+            if (y16)
+                y16[m * N + n] = qo_f64_to_f16(y);
+        }
+    return 0;
+}
+
 /* Nibble packing: byte i = code[2i] in bits 0-3, code[2i+1] in bits 4-7. */
 int qo_pack(const int8_t *codes, int64_t n, uint8_t *packed)
 {
