@@ -253,6 +253,58 @@ quarot_status_t quarot_rotate_quant_linear_i8(const void *x_f16, int64_t M, int6
                                               quarot_stream_t stream);
 
 /*
+ * ---------------------------------------------------------------------------
+ * Asymmetric INT4 with a clipping ratio [DQ-12: per-token asymmetric
+ * quantization of activations, per-channel asymmetric quantization of
+ * weights, clipping ratios on the extremes (0.9 for activations, 0.8 for
+ * weights in its setup), step (gamma max - beta min) / (2^b - 1)]:
+ *
+ *   per row of x' (rotated as in quarot_rotate_quant, full Hadamard):
+ *     lo = clip * min x', hi = clip * max x', d = (hi - lo) / 15 (fp32),
+ *     z = rint(-lo / d) (int32 zero point), u = clamp(rint(x'/d) + z, 0, 15),
+ *     reconstruction d * (u - z); a zero step gives zero codes and z = 0.
+ *   Codes u are unsigned nibbles packed two per byte (element 2i in bits 0-3).
+ *   The quantizer also returns the row's code sum r = sum_k u.
+ * The linear layer:
+ *   out[m,n] = fp16( d_a[m] d_w[n] (acc - z_w[n] r_a[m] - z_a[m] r_w[n] + K z_a[m] z_w[n]) ),
+ *   acc = sum_k u_a[m,k] u_w[n,k]  (int32, exact; the bracket is formed in 64-bit integers).
+ * ---------------------------------------------------------------------------
+ */
+
+/*
+ * quarot_rotate_quant_asym -- rotation + asymmetric 4-bit RTN of activations
+ * (per token) or, offline, of weight rows (per output channel).
+ * x_f16, signs, M, K: as quarot_rotate_quant; had_block must be 0 and
+ * 256 <= K <= 8192 (a power of two).  clip in (0, 1].
+ * q_packed [M, K/2] uint8, scales fp32 [M] (the steps d), zeros int32 [M],
+ * rowsums int32 [M]: outputs.  Valid while |z| < 2^22 (the clipped range
+ * of a row does not sit more than 2^22 steps away from zero).
+ */
+quarot_status_t quarot_rotate_quant_asym(const void *x_f16, int64_t M, int64_t K, const int8_t *signs,
+                                         int had_block, float clip, uint8_t *q_packed, float *scales,
+                                         int32_t *zeros, int32_t *rowsums, quarot_stream_t stream);
+
+/*
+ * quarot_uint4_gemm_s32 -- acc[m,n] = sum_k u_a[m,k] u_w[n,k] of unsigned
+ * nibble codes as int32 [M, N] (exact: acc <= 225 K).  Layouts and limits
+ * as quarot_int4_gemm_s32.  For testing the integer path in isolation.
+ */
+quarot_status_t quarot_uint4_gemm_s32(const uint8_t *qa, int64_t M, const uint8_t *qw, int64_t N, int64_t K,
+                                      int32_t *acc, quarot_stream_t stream);
+
+/*
+ * quarot_int4_linear_asym -- the asymmetric INT4 linear layer (formula
+ * above).  qa [M, K/2], s_a fp32 [M], z_a int32 [M], r_a int32 [M] (from
+ * quarot_rotate_quant_asym of the activations); qw [N, K/2], s_w, z_w, r_w
+ * [N] (the same call on the weight rows); out [M, N] fp16.
+ * Limits: as quarot_int4_linear with group 0.
+ */
+quarot_status_t quarot_int4_linear_asym(const uint8_t *qa, const float *s_a, const int32_t *z_a,
+                                        const int32_t *r_a, int64_t M, const uint8_t *qw, const float *s_w,
+                                        const int32_t *z_w, const int32_t *r_w, int64_t N, int64_t K,
+                                        void *out_f16, quarot_stream_t stream);
+
+/*
  * quarot_kv_quant -- INT4 KV-cache write [QR-A: the KV cache in 4 bits;
  * DQ-12: fixed Hadamard on the query-key product, per-head quantization].
  *

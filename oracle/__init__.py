@@ -44,6 +44,7 @@ def lib():
             "qo_quantize_bits": [P, I64, I64, ctypes.c_int, P, P],
             "qo_quantize_asym": [P, I64, I64, ctypes.c_int, ctypes.c_double, P, P, P, P],
             "qo_dequant_asym": [P, I64, I64, I64, P, P, P, P, P, P, P, P],
+            "qo_quantize_asym_with": [P, I64, I64, ctypes.c_int, P, P, P],
             "qo_quantize_bits_with_scales": [P, I64, I64, ctypes.c_int, P, P],
             "qo_pack": [P, I64, P],
             "qo_unpack": [P, I64, P],
@@ -214,6 +215,16 @@ def quantize_asym(xr, clip: float, bits: int = 4):
     _check(lib().qo_quantize_asym(_p(xr), M, K, bits, float(clip), _p(codes), _p(d), _p(z), _p(r)),
            "quantize_asym")
     return codes, d, z, r
+
+
+def quantize_asym_with(xr, step, zero, bits: int = 4) -> np.ndarray:
+    """Asymmetric RTN codes of xr [M, K] under given per-row steps and zero points."""
+    xr = _c(xr, np.float64)
+    M, K = xr.shape
+    codes = np.empty((M, K), np.int8)
+    _check(lib().qo_quantize_asym_with(_p(xr), M, K, bits, _p(_c(step, np.float64)), _p(_c(zero, np.int64)),
+                                       _p(codes)), "quantize_asym_with")
+    return codes
 
 
 def dequant_asym(acc, K, da, za, ra, dw, zw, rw):

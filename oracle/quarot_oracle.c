@@ -409,6 +409,30 @@ int qo_quantize_asym(const double *xr, int64_t M, int64_t K, int bits, double cl
     return 0;
 }
 
+/* The asymmetric RTN step alone under a caller-supplied step and zero point
+ * per row: u = clamp(rint(v / d) + z, 0, 2^bits - 1), zero step -> zero code. */
+int qo_quantize_asym_with(const double *xr, int64_t M, int64_t K, int bits, const double *step, const int64_t *zero,
+                          int8_t *codes)
+{
+    if (M < 0 || K <= 0 || bits < 2 || bits > 8)
+        return -1;
+    const double qmax = (double)((1 << bits) - 1);
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; ++r)
+        for (int64_t k = 0; k < K; ++k) {
+            double q = 0.0;
+            if (step[r] > 0.0) {
+                q = nearbyint(xr[r * K + k] / step[r]) + (double)zero[r];
+                if (q < 0.0)
+                    q = 0.0;
+                if (q > qmax)
+                    q = qmax;
+            }
+            codes[r * K + k] = (int8_t)q;
+        }
+    return 0;
+}
+
 /*
  * The dequantized product of asymmetric codes:
  *   y[m, n] = da[m] dw[n] sum_k (ua[m,k] - za[m]) (uw[n,k] - zw[n])

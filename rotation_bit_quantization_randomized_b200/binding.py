@@ -40,6 +40,9 @@ _SIGS = {
     "quarot_int8_gemm_s32": ([_P, _I64, _P, _I64, _I64, _P, _P], _INT),
     "quarot_rotate_quant_linear_i8_workspace": ([_I64, _I64], _SZ),
     "quarot_rotate_quant_linear_i8": ([_P, _I64, _I64, _P, _INT, _P, _P, _I64, _P, _SZ, _P, _P], _INT),
+    "quarot_rotate_quant_asym": ([_P, _I64, _I64, _P, _INT, ctypes.c_float, _P, _P, _P, _P, _P], _INT),
+    "quarot_uint4_gemm_s32": ([_P, _I64, _P, _I64, _I64, _P, _P], _INT),
+    "quarot_int4_linear_asym": ([_P, _P, _P, _P, _I64, _P, _P, _P, _P, _I64, _I64, _P, _P], _INT),
     "quarot_kv_quant": ([_P, _P, _I64, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P], _INT),
     "quarot_kv_decode_scores": ([_P, _I64, _I64, _P, _P, _P, _I64, _I64, _I64, _P, _P], _INT),
     "quarot_get_device_status": ([], _INT),
@@ -231,6 +234,45 @@ def quarot_rotate_quant_linear_i8(x: torch.Tensor, signs: torch.Tensor, qw: torc
            lib.quarot_rotate_quant_linear_i8(_ptr(x), M, K, _ptr(signs), had_block, _ptr(qw), _ptr(s_w), N,
                                              _ptr(workspace), workspace.numel() * workspace.element_size(),
                                              _ptr(out), _stream(stream)))
+    return out
+
+
+def quarot_rotate_quant_asym(x: torch.Tensor, signs: torch.Tensor, clip: float, had_block: int = 0, stream=None):
+    """x fp16 [M, K] -> (q_packed uint8 [M, K/2] unsigned nibbles, steps fp32 [M],
+    zero points int32 [M], code row sums int32 [M])."""
+    M, K = x.shape
+    dev = x.device
+    q = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+    d = torch.empty((M,), dtype=torch.float32, device=dev)
+    z = torch.empty((M,), dtype=torch.int32, device=dev)
+    r = torch.empty((M,), dtype=torch.int32, device=dev)
+    _check("quarot_rotate_quant_asym",
+           lib.quarot_rotate_quant_asym(_ptr(x), M, K, _ptr(signs), had_block, float(clip), _ptr(q), _ptr(d),
+                                        _ptr(z), _ptr(r), _stream(stream)))
+    return q, d, z, r
+
+
+def quarot_uint4_gemm_s32(qa: torch.Tensor, qw: torch.Tensor, acc: Optional[torch.Tensor] = None, stream=None):
+    """Exact int32 [M, N] = sum_k u_a u_w of unsigned nibble codes."""
+    M, Kh = qa.shape
+    N = qw.shape[0]
+    if acc is None:
+        acc = torch.empty((M, N), dtype=torch.int32, device=qa.device)
+    _check("quarot_uint4_gemm_s32",
+           lib.quarot_uint4_gemm_s32(_ptr(qa), M, _ptr(qw), N, 2 * Kh, _ptr(acc), _stream(stream)))
+    return acc
+
+
+def quarot_int4_linear_asym(qa, s_a, z_a, r_a, qw, s_w, z_w, r_w, out: Optional[torch.Tensor] = None,
+                            stream=None):
+    """The asymmetric INT4 linear layer -> fp16 [M, N]."""
+    M, Kh = qa.shape
+    N = qw.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=qa.device)
+    _check("quarot_int4_linear_asym",
+           lib.quarot_int4_linear_asym(_ptr(qa), _ptr(s_a), _ptr(z_a), _ptr(r_a), M, _ptr(qw), _ptr(s_w), _ptr(z_w),
+                                       _ptr(r_w), N, 2 * Kh, _ptr(out), _stream(stream)))
     return out
 
 

@@ -162,6 +162,32 @@ __device__ __forceinline__ void fma_x2_acc(float a0, float a1, float b, float &a
         : "f"(a0), "f"(a1), "f"(b));
 }
 
+// min(a, b, c): the three-input form of sm_100 (one instruction).
+__device__ __forceinline__ float min3f(float a, float b, float c)
+{
+    float r;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+__device__ __forceinline__ float warp_min(float v, int width)
+{
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1)
+        if (o < width)
+            v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t warp_sum(uint32_t v, int width)
+{
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1)
+        if (o < width)
+            v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
 __device__ __forceinline__ float warp_max(float v, int width)
 {
 #pragma unroll

@@ -46,7 +46,7 @@
 
 namespace quarot {
 
-enum : int { kEpiScaledF16 = 0, kEpiS32 = 1, kEpiGroupF16 = 2 };
+enum : int { kEpiScaledF16 = 0, kEpiS32 = 1, kEpiGroupF16 = 2, kEpiAsymF16 = 3 };
 
 constexpr int kGemmBM = 128;
 constexpr int kGemmBK = 128;            // int8 elements of K per stage (one 128-byte row)
@@ -96,6 +96,8 @@ struct GemmArgs {
     const uint8_t *qw;      // [N, K/2]
     const void *sw;         // fp32 [N] or fp16 [N, K/128]
     void *out;              // fp16 or int32 [M, N]
+    const int32_t *za, *ra; // asymmetric: activation zero points and code row sums [M]
+    const int32_t *zw, *rw; // asymmetric: weight zero points and code row sums [N]
     int64_t M, N, K;
     int tiles_m, tiles_n, kblocks;
 };

@@ -88,7 +88,9 @@ struct PairShape {
                   "each stage barrier is used by one unpack group");
 };
 
-template <int BN, int EPI>
+// UNS: the codes are unsigned nibbles (asymmetric quantization): they are
+// widened to the byte values 0..15 and multiplied as unsigned 8-bit.
+template <int BN, int EPI, bool UNS = false>
 __global__ void __launch_bounds__(PairShape<BN, EPI>::kThreads, 1)
 int4_gemm_pair_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_a,
                       const __grid_constant__ CUtensorMap tma_b)
@@ -219,8 +221,8 @@ int4_gemm_pair_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_
                 const uint32_t w4[4] = {wa[c].x, wa[c].y, wa[c].z, wa[c].w};
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    av[8 * c + i] = (w4[i] << 4) & 0xF0F0F0F0u;
-                    av[8 * c + 4 + i] = w4[i] & 0xF0F0F0F0u;
+                    av[8 * c + i] = UNS ? (w4[i] & 0x0F0F0F0Fu) : ((w4[i] << 4) & 0xF0F0F0F0u);
+                    av[8 * c + 4 + i] = UNS ? ((w4[i] >> 4) & 0x0F0F0F0Fu) : (w4[i] & 0xF0F0F0F0u);
                 }
             }
             // B stage bs is free once the MMAs of step - kBStages are done
@@ -234,10 +236,14 @@ int4_gemm_pair_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_
                     const int r = 8 * g + rsub;
                     uint8_t *dst = st_base + g * 1024 + rsub * 128;
                     const uint4 v = wb[j];
-                    const uint4 lo = make_uint4((v.x << 4) & 0xF0F0F0F0u, (v.y << 4) & 0xF0F0F0F0u,
-                                                (v.z << 4) & 0xF0F0F0F0u, (v.w << 4) & 0xF0F0F0F0u);
-                    const uint4 hi = make_uint4(v.x & 0xF0F0F0F0u, v.y & 0xF0F0F0F0u, v.z & 0xF0F0F0F0u,
-                                                v.w & 0xF0F0F0F0u);
+                    const uint4 lo = UNS ? make_uint4(v.x & 0x0F0F0F0Fu, v.y & 0x0F0F0F0Fu, v.z & 0x0F0F0F0Fu,
+                                                      v.w & 0x0F0F0F0Fu)
+                                         : make_uint4((v.x << 4) & 0xF0F0F0F0u, (v.y << 4) & 0xF0F0F0F0u,
+                                                      (v.z << 4) & 0xF0F0F0F0u, (v.w << 4) & 0xF0F0F0F0u);
+                    const uint4 hi = UNS ? make_uint4((v.x >> 4) & 0x0F0F0F0Fu, (v.y >> 4) & 0x0F0F0F0Fu,
+                                                      (v.z >> 4) & 0x0F0F0F0Fu, (v.w >> 4) & 0x0F0F0F0Fu)
+                                         : make_uint4(v.x & 0xF0F0F0F0u, v.y & 0xF0F0F0F0u, v.z & 0xF0F0F0F0u,
+                                                      v.w & 0xF0F0F0F0u);
                     *reinterpret_cast<uint4 *>(dst + (((2 * csub) ^ (r & 7)) << 4)) = lo;
                     *reinterpret_cast<uint4 *>(dst + (((2 * csub + 1) ^ (r & 7)) << 4)) = hi;
                 }
@@ -270,7 +276,7 @@ int4_gemm_pair_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_
     } else if (warp == S::kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer (leader only)
         if (leader && lane == 0) {
-            constexpr uint32_t idesc = idesc_i8(kPairBM, BN);
+            constexpr uint32_t idesc = idesc_i8(kPairBM, BN, UNS);
             bool ok = true;
             int step = 0;
             for (int lt = 0; lt < my_tiles && ok; ++lt) {
@@ -316,8 +322,14 @@ int4_gemm_pair_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_
                 break;
             tc_fence_after();
             float sam = 0.f;
+            int32_t zam = 0, ram = 0;
             if (EPI == kEpiScaledF16 && mrow)
                 sam = reinterpret_cast<const float *>(a.sa)[m] * (1.0f / 256.0f);
+            if (EPI == kEpiAsymF16 && mrow) {
+                sam = reinterpret_cast<const float *>(a.sa)[m];
+                zam = a.za[m];
+                ram = a.ra[m];
+            }
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t r[32];
@@ -350,15 +362,52 @@ int4_gemm_pair_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_
                             *reinterpret_cast<uint4 *>(orow + n) = make_uint4(h[0], h[1], h[2], h[3]);
                         }
                     }
+                } else if (mrow && EPI == kEpiAsymF16) {
+                    // y = da dw (acc - zw ra - za rw + K za zw): the bracket is formed
+                    // exactly in 64-bit integers (zero points are not bounded by the
+                    // code width), then converted and scaled
+                    __half *orow = reinterpret_cast<__half *>(a.out) + m * a.N;
+                    const float *swp = reinterpret_cast<const float *>(a.sw);
+                    const int64_t kz = a.K * (int64_t)zam;
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        const int64_t n = n0 + 32 * c + 8 * v;
+                        if (n < a.N) {
+                            const float4 w0 = __ldg(reinterpret_cast<const float4 *>(swp + n));
+                            const float4 w1 = __ldg(reinterpret_cast<const float4 *>(swp + n + 4));
+                            const int4 z0 = __ldg(reinterpret_cast<const int4 *>(a.zw + n));
+                            const int4 z1 = __ldg(reinterpret_cast<const int4 *>(a.zw + n + 4));
+                            const int4 s0 = __ldg(reinterpret_cast<const int4 *>(a.rw + n));
+                            const int4 s1 = __ldg(reinterpret_cast<const int4 *>(a.rw + n + 4));
+                            const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                            const int32_t zv[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+                            const int32_t sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+                            uint32_t h[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                float f[2];
+#pragma unroll
+                                for (int e = 0; e < 2; ++e) {
+                                    const int k = 2 * i + e;
+                                    const int64_t br = (int64_t)(int32_t)r[8 * v + k] - (int64_t)zv[k] * ram -
+                                                       (int64_t)zam * sv[k] + kz * zv[k];
+                                    f[e] = __ll2float_rn(br) * sam * wv[k];
+                                }
+                                h[i] = h2_as_u32(__floats2half2_rn(f[0], f[1]));
+                            }
+                            *reinterpret_cast<uint4 *>(orow + n) = make_uint4(h[0], h[1], h[2], h[3]);
+                        }
+                    }
                 } else if (mrow) {
                     int32_t *orow = reinterpret_cast<int32_t *>(a.out) + m * a.N;
+                    constexpr int sh = UNS ? 0 : 8;           // signed codes are widened x16 each
 #pragma unroll
                     for (int v = 0; v < 8; ++v) {
                         const int64_t n = n0 + 32 * c + 4 * v;
                         if (n < a.N)
                             *reinterpret_cast<int4 *>(orow + n) =
-                                make_int4((int)r[4 * v] >> 8, (int)r[4 * v + 1] >> 8, (int)r[4 * v + 2] >> 8,
-                                          (int)r[4 * v + 3] >> 8);
+                                make_int4((int)r[4 * v] >> sh, (int)r[4 * v + 1] >> sh, (int)r[4 * v + 2] >> sh,
+                                          (int)r[4 * v + 3] >> sh);
                     }
                 }
             }

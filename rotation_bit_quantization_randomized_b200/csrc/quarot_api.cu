@@ -149,11 +149,11 @@ quarot_status_t check_rotate_args(const void *x, int64_t M, int64_t K, const int
 // qmax of a code width: the largest code magnitude of the symmetric RTN.
 constexpr double qmax_of(int bits) { return bits == 8 ? 127.0 : 7.0; }
 
-template <int LOGN, int GROUP, int BITS>
+template <int LOGN, int GROUP, int BITS, bool ASYM = false>
 quarot_status_t launch_fwht(const void *x, int64_t M, const int8_t *signs, uint8_t *q, void *scales,
-                            cudaStream_t st, int dev, int sms)
+                            cudaStream_t st, int dev, int sms, AsymOut asym = AsymOut{nullptr, nullptr, 1.0f})
 {
-    auto kern = fwht_quant_kernel<LOGN, GROUP, BITS>;
+    auto kern = fwht_quant_kernel<LOGN, GROUP, BITS, ASYM>;
     constexpr int smem = FwhtSmem<LOGN>::kBytes;
     int per_sm = 0;
     quarot_status_t s = kernel_occupancy(kern, dev, kFwhtThreads, smem, per_sm);
@@ -163,8 +163,9 @@ quarot_status_t launch_fwht(const void *x, int64_t M, const int8_t *signs, uint8
     const int64_t ctas = (M + R - 1) / R;
     const int grid = (int)std::min<int64_t>(ctas, (int64_t)sms * per_sm);
     const double n = double(1 << LOGN);
-    kern<<<grid, kFwhtThreads, smem, st>>>(reinterpret_cast<const uint32_t *>(x), M, signs, q, scales,
-                                        (float)(1.0 / (qmax_of(BITS) * std::sqrt(n))), (float)std::sqrt(n));
+    const double mul = ASYM ? 1.0 / std::sqrt(n) : 1.0 / (qmax_of(BITS) * std::sqrt(n));
+    kern<<<grid, kFwhtThreads, smem, st>>>(reinterpret_cast<const uint32_t *>(x), M, signs, q, scales, (float)mul,
+                                           (float)std::sqrt(n), asym);
     return after_launch("fwht_quant_kernel launch");
 }
 
@@ -179,6 +180,21 @@ quarot_status_t dispatch_fwht(int logn, const void *x, int64_t M, const int8_t *
     case 11: return launch_fwht<11, GROUP, BITS>(x, M, signs, q, scales, st, dev, sms);
     case 12: return launch_fwht<12, GROUP, BITS>(x, M, signs, q, scales, st, dev, sms);
     case 13: return launch_fwht<13, GROUP, BITS>(x, M, signs, q, scales, st, dev, sms);
+    default: return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "unsupported transform size");
+    }
+}
+
+// The asymmetric quantizer (full transform, K a power of two in [256, 8192]).
+quarot_status_t dispatch_fwht_asym(int logn, const void *x, int64_t M, const int8_t *signs, uint8_t *q,
+                                   float *scales, AsymOut asym, cudaStream_t st, int dev, int sms)
+{
+    switch (logn) {
+    case 8: return launch_fwht<8, 0, 4, true>(x, M, signs, q, scales, st, dev, sms, asym);
+    case 9: return launch_fwht<9, 0, 4, true>(x, M, signs, q, scales, st, dev, sms, asym);
+    case 10: return launch_fwht<10, 0, 4, true>(x, M, signs, q, scales, st, dev, sms, asym);
+    case 11: return launch_fwht<11, 0, 4, true>(x, M, signs, q, scales, st, dev, sms, asym);
+    case 12: return launch_fwht<12, 0, 4, true>(x, M, signs, q, scales, st, dev, sms, asym);
+    case 13: return launch_fwht<13, 0, 4, true>(x, M, signs, q, scales, st, dev, sms, asym);
     default: return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "unsupported transform size");
     }
 }
@@ -348,8 +364,9 @@ quarot_status_t launch_gemm(GemmArgs a, cudaStream_t st, bool pdl)
 // tensor memory for two A stages.
 constexpr int kPairBN = 224;
 
-// The per-token / per-channel GEMM on CTA pairs (clusters of two).
-template <int EPI>
+// The per-token / per-channel GEMM on CTA pairs (clusters of two); UNS for
+// unsigned (asymmetric) codes.
+template <int EPI, bool UNS = false>
 quarot_status_t launch_gemm_pair(GemmArgs a, cudaStream_t st, bool pdl)
 {
     using S = PairShape<kPairBN, EPI>;
@@ -358,7 +375,7 @@ quarot_status_t launch_gemm_pair(GemmArgs a, cudaStream_t st, bool pdl)
     quarot_status_t s = current_device(dev, info);
     if (s != QUAROT_OK)
         return s;
-    auto kern = int4_gemm_pair_kernel<kPairBN, EPI>;
+    auto kern = int4_gemm_pair_kernel<kPairBN, EPI, UNS>;
     int per_sm = 0;
     s = kernel_occupancy(kern, dev, S::kThreads, S::kSmemBytes, per_sm);
     if (s != QUAROT_OK)
@@ -747,6 +764,76 @@ quarot_status_t quarot_rotate_quant_linear_i8(const void *x_f16, int64_t M, int6
     if (s != QUAROT_OK)
         return s;
     return linear8_launch(qa, sa, M, qw, s_w, N, K, out_f16, st, true);
+}
+
+quarot_status_t quarot_rotate_quant_asym(const void *x_f16, int64_t M, int64_t K, const int8_t *signs, int had_block,
+                                         float clip, uint8_t *q_packed, float *scales, int32_t *zeros,
+                                         int32_t *rowsums, quarot_stream_t stream)
+{
+    quarot_status_t s = check_rotate_args(x_f16, M, K, signs, had_block, 0, q_packed, scales);
+    if (s != QUAROT_OK)
+        return s;
+    if (!(clip > 0.0f) || clip > 1.0f)
+        return fail(QUAROT_ERR_INVALID_ARG, "clip must lie in (0, 1]");
+    if (had_block != 0 || K < 256)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "asymmetric quantization needs the full Hadamard, 256 <= K <= 8192");
+    if (M == 0)
+        return QUAROT_OK;
+    if (!zeros || !rowsums)
+        return fail(QUAROT_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(zeros) || !aligned16(rowsums))
+        return fail(QUAROT_ERR_MISALIGNED, "zeros and rowsums must be 16-byte aligned");
+    int dev;
+    DeviceInfo *info;
+    s = current_device(dev, info);
+    if (s != QUAROT_OK)
+        return s;
+    return dispatch_fwht_asym(ilog2(K), x_f16, M, signs, q_packed, scales, AsymOut{zeros, rowsums, clip},
+                              (cudaStream_t)stream, dev, info->sm_count);
+}
+
+quarot_status_t quarot_uint4_gemm_s32(const uint8_t *qa, int64_t M, const uint8_t *qw, int64_t N, int64_t K,
+                                      int32_t *acc, quarot_stream_t stream)
+{
+    quarot_status_t s = check_gemm_args(qa, M, qw, N, K, acc, nullptr, nullptr, false);
+    if (s != QUAROT_OK || M == 0)
+        return s;
+    GemmArgs a = {};
+    a.qa = qa;
+    a.qw = qw;
+    a.out = acc;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    return launch_gemm_pair<kEpiS32, true>(a, (cudaStream_t)stream, false);
+}
+
+quarot_status_t quarot_int4_linear_asym(const uint8_t *qa, const float *s_a, const int32_t *z_a, const int32_t *r_a,
+                                        int64_t M, const uint8_t *qw, const float *s_w, const int32_t *z_w,
+                                        const int32_t *r_w, int64_t N, int64_t K, void *out_f16,
+                                        quarot_stream_t stream)
+{
+    quarot_status_t s = check_gemm_args(qa, M, qw, N, K, out_f16, s_a, s_w, true);
+    if (s != QUAROT_OK || M == 0)
+        return s;
+    if (!z_a || !r_a || !z_w || !r_w)
+        return fail(QUAROT_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(z_a) || !aligned16(r_a) || !aligned16(z_w) || !aligned16(r_w))
+        return fail(QUAROT_ERR_MISALIGNED, "zero points and code sums must be 16-byte aligned");
+    GemmArgs a = {};
+    a.qa = qa;
+    a.sa = s_a;
+    a.za = z_a;
+    a.ra = r_a;
+    a.qw = qw;
+    a.sw = s_w;
+    a.zw = z_w;
+    a.rw = r_w;
+    a.out = out_f16;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    return launch_gemm_pair<kEpiAsymF16, true>(a, (cudaStream_t)stream, false);
 }
 
 quarot_status_t quarot_kv_quant(const void *k_f16, const void *v_f16, int64_t B, int64_t T, int64_t Hkv, int64_t D,

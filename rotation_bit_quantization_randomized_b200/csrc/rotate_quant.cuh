@@ -80,6 +80,49 @@ __device__ __forceinline__ void quant_pack_store(const float (&v)[128], float r,
     }
 }
 
+// Asymmetric 4-bit codes of 128 values of one thread (packed as usual) and
+// their sum.  cz = 1.5 * 2^23 + z (z the integer zero point), r = 1 / step:
+// fma(v, r, cz) holds rint(v r) + z in its low mantissa bits, clamped in
+// float to [0, 15] before the nibble is taken.
+__device__ __forceinline__ uint32_t quant_pack_store_asym(const float (&v)[128], float r, float cz, uint8_t *dst,
+                                                          bool valid)
+{
+    constexpr float C = 12582912.0f;
+    uint32_t pk[16];
+    uint32_t sum = 0;
+#pragma unroll
+    for (int g = 0; g < 16; ++g) {
+        uint32_t acc = 0;
+#pragma unroll
+        for (int k = 0; k < 8; k += 2) {
+            float f0, f1;
+            fma_x2(v[8 * g + k], v[8 * g + k + 1], r, cz, f0, f1);
+            f0 = fminf(fmaxf(f0, C), C + 15.0f);
+            f1 = fminf(fmaxf(f1, C), C + 15.0f);
+            acc = push_nibble(acc, __float_as_uint(f0));
+            acc = push_nibble(acc, __float_as_uint(f1));
+        }
+        pk[g] = acc;
+        // the eight nibbles of acc: pairwise byte sums, then the byte total
+        const uint32_t b = (acc & 0x0F0F0F0Fu) + ((acc >> 4) & 0x0F0F0F0Fu);
+        sum += (b * 0x01010101u) >> 24;
+    }
+    if (valid) {
+        uint4 *d = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            d[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+    }
+    return sum;
+}
+
+// Outputs of the asymmetric quantizer beyond codes and steps.
+struct AsymOut {
+    int32_t *zeros;      // [M] zero points
+    int32_t *rowsums;    // [M] sums of the row's codes
+    float clip;          // clipping ratio of the row's min and max
+};
+
 // Rounds 128 values of one thread to signed 8-bit codes and stores the 128
 // bytes (the 8-bit variant of the same RTN).  r = 127 / max|y| of the row, so
 // |v r| <= 127 (1 + 2^-23) and no clamp is needed; the low byte of the bit
@@ -135,21 +178,23 @@ struct FwhtSmem {
     static constexpr int kRowFloats = (N / 128) * kChunk + (LOGN == 10 ? 8 : 4);
     static constexpr int kBufOffset = kStageBytes;
     static constexpr int kBarOffset = kBufOffset + R * kRowFloats * 4;
-    static constexpr int kBytes = kBarOffset + 16 + 16;
+    static constexpr int kBytes = kBarOffset + 16 + 32;   // mbarrier, then 8 reduction words
     static_assert(kStageRowBytes % 16 == 0 && kBufOffset % 16 == 0, "16-byte aligned staging and buffer");
 };
 
-template <int LOGN, int GROUP, int BITS = 4>
+template <int LOGN, int GROUP, int BITS = 4, bool ASYM = false>
 __global__ void __launch_bounds__(kFwhtThreads, 4)
 fwht_quant_kernel(const uint32_t *__restrict__ x,      // [M, K/2] fp16 pairs
                   int64_t M, const int8_t *__restrict__ signs,
                   uint8_t *__restrict__ q,             // [M, K/2] (4-bit) or [M, K] (8-bit)
                   void *__restrict__ scales,           // fp32 [M] or fp16 [M, K/128]
-                  float scale_mul,                     // 1 / (qmax sqrt(K)), rounded to fp32
-                  float sqrt_n)                        // sqrt(K), rounded to fp32
+                  float scale_mul,                     // 1 / (qmax sqrt(K)) (asymmetric: 1 / sqrt(K))
+                  float sqrt_n,                        // sqrt(K), rounded to fp32
+                  AsymOut asym)                        // asymmetric variant only
 {
     static_assert(LOGN >= 8 && LOGN <= 13, "full transform covers 256..8192");
     static_assert(BITS == 4 || (BITS == 8 && GROUP == 0), "8-bit codes use one scale per row");
+    static_assert(!ASYM || (GROUP == 0 && BITS == 4), "asymmetric codes: 4 bits, one step per row");
     using S = FwhtSmem<LOGN>;
     constexpr float kQmax = BITS == 8 ? 127.0f : 7.0f;
     constexpr int N = S::N;
@@ -253,6 +298,53 @@ fwht_quant_kernel(const uint32_t *__restrict__ x,      // [M, K/2] fp16 pairs
 #pragma unroll
         for (int i = 0; i < 128; i += 2)
             amax = max3f(amax, fabsf(v[i]), fabsf(v[i + 1]));
+
+        if (ASYM) {
+            // per-row min and max, clipped range, step, zero point; then the
+            // codes and the row's code sum
+            float amx = v[0], amn = v[0];
+#pragma unroll
+            for (int i = 0; i < 128; i += 2) {
+                amx = max3f(amx, v[i], v[i + 1]);
+                amn = min3f(amn, v[i], v[i + 1]);
+            }
+            if (T <= 32) {
+                amx = warp_max(amx, T);
+                amn = warp_min(amn, T);
+                __syncthreads();                      // buffer reads done before reuse
+            } else {
+                amx = warp_max(amx, 32);
+                amn = warp_min(amn, 32);
+                if ((tid & 31) == 0) {
+                    red[tid >> 5] = amx;
+                    red[2 + (tid >> 5)] = amn;
+                }
+                __syncthreads();
+                amx = fmaxf(red[0], red[1]);
+                amn = fminf(red[2], red[3]);
+            }
+            const float lo = asym.clip * amn, hi = asym.clip * amx;
+            const float dv = (hi - lo) / 15.0f;
+            const float z = dv > 0.f ? rintf(-lo / dv) : 0.f;
+            const float r = dv > 0.f ? 1.0f / dv : 0.f;
+            uint32_t csum = quant_pack_store_asym(v, r, 12582912.0f + z, q + (valid ? row : 0) * (N / 2) + tr * 64,
+                                                  valid);
+            if (T <= 32) {
+                csum = warp_sum(csum, T);
+            } else {
+                csum = warp_sum(csum, 32);
+                if ((tid & 31) == 0)
+                    reinterpret_cast<uint32_t *>(red)[4 + (tid >> 5)] = csum;
+                __syncthreads();
+                csum = reinterpret_cast<uint32_t *>(red)[4] + reinterpret_cast<uint32_t *>(red)[5];
+            }
+            if (valid && tr == 0) {
+                reinterpret_cast<float *>(scales)[row] = dv * scale_mul;
+                asym.zeros[row] = (int32_t)z;
+                asym.rowsums[row] = (int32_t)csum;
+            }
+            continue;
+        }
 
         float r;
         if (GROUP == 0) {

@@ -296,10 +296,11 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr)
 }
 
 // Instruction descriptor for kind::i8: s32 accumulator, both operands signed
-// 8-bit and K-major, M x N tile.
-__host__ __device__ constexpr uint32_t idesc_i8(int M, int N)
+// (or, with is_unsigned, both unsigned) 8-bit and K-major, M x N tile.
+__host__ __device__ constexpr uint32_t idesc_i8(int M, int N, bool is_unsigned = false)
 {
-    return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+    return (2u << 4) | ((is_unsigned ? 0u : 1u) << 7) | ((is_unsigned ? 0u : 1u) << 10) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 }  // namespace quarot

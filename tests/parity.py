@@ -133,3 +133,45 @@ def check_codes_bits(gpu_codes, gpu_scales, xr, bits, max_frac=1e-4):
     counted = int((flips & ~exact_tie).sum())
     assert counted <= max_frac * got.size, f"{counted} near-tie code flips in {got.size} elements"
     return n
+
+
+def check_codes_asym(gpu_packed, gpu_step, gpu_zero, gpu_rowsum, xr, clip, max_frac=1e-4):
+    """Rules for the asymmetric 4-bit quantizer (per row: step from the clipped
+    min/max, zero point, unsigned codes, code sum).
+     * step within 1e-6 relative of the oracle's fp64 step;
+     * zero point equal to the oracle's, or one away only where the oracle's
+       -lo/step lies within 1e-4 of a rounding boundary (both are correct
+       roundings of a near-tie);
+     * codes: the oracle's RTN under the device's step and zero point, +-1
+       only within 1e-3 of a rounding boundary, at most max_frac of elements
+       (exact ties excluded, as in the symmetric rule);
+     * the code sum equals the sum of the device's own codes."""
+    M, K = xr.shape
+    u_o, d_o, z_o, _ = oracle.quantize_asym(xr, clip)
+    d = np.asarray(gpu_step, np.float64)
+    z = np.asarray(gpu_zero, np.int64)
+    rel = np.abs(d - d_o) / np.maximum(d_o, 1e-300)
+    bad = (rel > 1e-6) & ~((d_o == 0) & (d == 0))
+    assert not np.any(bad), f"steps off: max rel {rel[bad].max():.3e}"
+    dz = z - z_o
+    if np.any(dz != 0):
+        assert np.all(np.abs(dz[dz != 0]) == 1), "zero points more than one away"
+        lo = clip * xr.min(axis=1)
+        t = np.where(d_o > 0, -lo / np.where(d_o > 0, d_o, 1.0), 0.0)
+        dist = np.abs(t - (np.floor(t) + 0.5))
+        assert np.all(dist[dz != 0] < 1e-4), "zero point differs away from a rounding near-tie"
+    got = (oracle.unpack(np.asarray(gpu_packed, np.uint8)) & 0x0F).astype(np.int64).reshape(M, K)
+    np.testing.assert_array_equal(got.sum(axis=1), np.asarray(gpu_rowsum, np.int64))
+    expect = oracle.quantize_asym_with(xr, d, z).astype(np.int64)
+    diff = got - expect
+    flips = diff != 0
+    if not np.any(flips):
+        return 0
+    assert np.all(np.abs(diff[flips]) == 1), "codes differ by more than one step"
+    t = np.where(d[:, None] > 0, xr / np.where(d[:, None] > 0, d[:, None], 1.0), 0.0)
+    dist = np.abs(t - (np.floor(t) + 0.5))
+    assert np.all(dist[flips] < 1e-3), f"code flips away from near-ties (max dist {dist[flips].max():.3e})"
+    exact_tie = dist <= 1e-9 * np.maximum(1.0, np.abs(t))
+    counted = int((flips & ~exact_tie).sum())
+    assert counted <= max_frac * got.size, f"{counted} near-tie code flips in {got.size} elements"
+    return int(flips.sum())

@@ -102,3 +102,12 @@ def test_linear_asym_error_bound_tiny_workload():
 def test_clip_ratio_range_is_checked(bad):
     with pytest.raises(ValueError):
         oracle.quantize_asym(np.ones((1, 4)), bad)
+
+
+def test_quantize_asym_with_own_step_and_zero_reproduces_codes_and_hand_values():
+    x = synth.random_f16((16, 256), 23, dist="laplace").astype(np.float64)
+    u, d, z, r = oracle.quantize_asym(x, 0.9)
+    np.testing.assert_array_equal(oracle.quantize_asym_with(x, d, z), u)
+    # hand values: d = 0.5, z = 3: x/d = -10, -1.5 (even -> -2), 0.6, 30 -> +3, clamp
+    got = oracle.quantize_asym_with(np.array([[-5.0, -0.75, 0.3, 15.0]]), np.array([0.5]), np.array([3]))
+    np.testing.assert_array_equal(got[0], [0, 1, 4, 15])
