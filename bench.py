@@ -46,8 +46,8 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--cpu-rows", type=int, default=2048, help="token rows of the CPU-baseline sample")
-    p.add_argument("--case", choices=["gemm", "gemm_group", "gemm8", "gemm8_full", "rotate", "block", "kvquant",
-                                      "kvscores"],
+    p.add_argument("--case", choices=["gemm", "gemm_group", "gemm8", "gemm8_full", "gemm_asym", "rotate",
+                                      "rotate_asym", "block", "kvquant", "kvscores"],
                    default=None, help="time one kernel on a capture-sized workload (for ncu), not the step")
     return p.parse_args()
 
@@ -427,6 +427,26 @@ def run_case(args):
         out = torch.empty((M, N), dtype=torch.float16, device=dev)
         fn = lambda: q.quarot_int8_linear(qa, sa, qw, sw, out)
         work, unit = 2.0 * M * N * K / 1e12, "TOPS"
+    elif args.case == "gemm_asym":
+        M, N, K = 4096, 28672, 8192
+        qa = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=dev, generator=g)
+        qw = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=dev, generator=g)
+        sa = torch.rand((M,), device=dev, generator=g) + 0.5
+        sw = torch.rand((N,), device=dev, generator=g) * 1e-3 + 1e-3
+        za = torch.randint(6, 10, (M,), dtype=torch.int32, device=dev, generator=g)
+        zw = torch.randint(6, 10, (N,), dtype=torch.int32, device=dev, generator=g)
+        ra = torch.randint(0, 15 * K, (M,), dtype=torch.int32, device=dev, generator=g)
+        rw = torch.randint(0, 15 * K, (N,), dtype=torch.int32, device=dev, generator=g)
+        out = torch.empty((M, N), dtype=torch.float16, device=dev)
+        fn = lambda: q.quarot_int4_linear_asym(qa, sa, za, ra, qw, sw, zw, rw, out)
+        work, unit = 2.0 * M * N * K / 1e12, "TOPS"
+    elif args.case == "rotate_asym":
+        M, K = 8192, 8192
+        x = torch.randn((M, K), device=dev, generator=g).half()
+        s = (torch.randint(0, 2, (K,), device=dev, generator=g) * 2 - 1).to(torch.int8)
+        outs = q.quarot_rotate_quant_asym(x, s, 0.9)
+        fn = lambda: q.quarot_rotate_quant_asym(x, s, 0.9, 0, *outs)
+        work, unit = bytes_rotate_quant(M, K) / 1e9, "GB/s"
     elif args.case in ("rotate", "block"):
         M, K = (8192, 8192) if args.case == "rotate" else (8192, 11008)
         hb, group = (0, 0) if args.case == "rotate" else (128, 128)

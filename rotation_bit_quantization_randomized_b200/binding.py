@@ -237,15 +237,16 @@ def quarot_rotate_quant_linear_i8(x: torch.Tensor, signs: torch.Tensor, qw: torc
     return out
 
 
-def quarot_rotate_quant_asym(x: torch.Tensor, signs: torch.Tensor, clip: float, had_block: int = 0, stream=None):
+def quarot_rotate_quant_asym(x: torch.Tensor, signs: torch.Tensor, clip: float, had_block: int = 0, q=None, d=None,
+                             z=None, r=None, stream=None):
     """x fp16 [M, K] -> (q_packed uint8 [M, K/2] unsigned nibbles, steps fp32 [M],
-    zero points int32 [M], code row sums int32 [M])."""
+    zero points int32 [M], code row sums int32 [M]); outputs may be passed in."""
     M, K = x.shape
     dev = x.device
-    q = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
-    d = torch.empty((M,), dtype=torch.float32, device=dev)
-    z = torch.empty((M,), dtype=torch.int32, device=dev)
-    r = torch.empty((M,), dtype=torch.int32, device=dev)
+    q = torch.empty((M, K // 2), dtype=torch.uint8, device=dev) if q is None else q
+    d = torch.empty((M,), dtype=torch.float32, device=dev) if d is None else d
+    z = torch.empty((M,), dtype=torch.int32, device=dev) if z is None else z
+    r = torch.empty((M,), dtype=torch.int32, device=dev) if r is None else r
     _check("quarot_rotate_quant_asym",
            lib.quarot_rotate_quant_asym(_ptr(x), M, K, _ptr(signs), had_block, float(clip), _ptr(q), _ptr(d),
                                         _ptr(z), _ptr(r), _stream(stream)))
