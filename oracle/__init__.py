@@ -52,6 +52,7 @@ def lib():
             "qo_dequant_linear": [P, I64, I64, I64, P, P, P, P],
             "qo_kv_quant": [P, P, I64, I64, I64, I64, P, P, P, P, P],
             "qo_kv_scores": [P, I64, I64, I64, I64, I64, P, P, P, P],
+            "qo_kv_attend": [P, I64, I64, I64, I64, I64, P, P, P],
             "qo_f16_to_f64_array": [P, I64, P],
             "qo_f64_to_f16_array": [P, I64, P],
             "qo_max_threads": [],
@@ -373,4 +374,18 @@ def kv_scores(q16, signs, kq_packed, ks):
     out = np.empty((B, Hq, T), np.float64)
     _check(lib().qo_kv_scores(_p(qb), B, Hq, H, D, T, _p(s), _p(kc), _p(ks64), _p(out)),
            "kv_scores")
+    return out
+
+
+def kv_attend(scores, vq_packed, vs):
+    """scores [B, Hq, T] (any float); vq_packed [B, T, H, D/2]; vs fp16 bits [B, T, H]
+    -> fp64 [B, Hq, D]: softmax(scores / sqrt(D)) over T times the dequantized values."""
+    sc = _c(np.asarray(scores, np.float64), np.float64)
+    B, Hq, T = sc.shape
+    vc = unpack(vq_packed)
+    _, T2, H, D = vc.shape
+    assert T2 == T
+    vs64 = _c(scales_to_f64(vs), np.float64)
+    out = np.empty((B, Hq, D), np.float64)
+    _check(lib().qo_kv_attend(_p(sc), B, Hq, H, D, T, _p(vc), _p(vs64), _p(out)), "kv_attend")
     return out

@@ -607,6 +607,48 @@ int qo_kv_scores(const uint16_t *q16, int64_t B, int64_t Hq, int64_t H, int64_t 
     return 0;
 }
 
+/*
+ * The rest of one decode step of attention over the INT4 value cache
+ * (QuaRot abstract: the KV cache in 4 bits, the attention path rotated too;
+ * DuQuant Knowl 12: the attention output x value product runs on quantized
+ * values while the softmax outputs stay unquantized):
+ *   p[b,hq,t] = softmax over t of scores[b,hq,t] / sqrt(D),
+ *   out[b,hq,d] = sum_t p[b,hq,t] * vscale[b,t,h] * vcode[b,t,h,d],  h = hq / (Hq/H).
+ * The value rows were not rotated, so no inverse rotation follows.  The
+ * softmax subtracts the row maximum before exponentiating (the same
+ * function, evaluated without overflow).
+ */
+int qo_kv_attend(const double *scores, int64_t B, int64_t Hq, int64_t H, int64_t D, int64_t T,
+                 const int8_t *vcodes, const double *vscale, double *out)
+{
+    if (D <= 0 || H <= 0 || Hq % H != 0 || B < 0 || T <= 0)
+        return -1;
+    int64_t grp = Hq / H;
+#pragma omp parallel for schedule(static)
+    for (int64_t bh = 0; bh < B * Hq; ++bh) {
+        int64_t b = bh / Hq, hq = bh % Hq, h = hq / grp;
+        const double *sr = scores + (b * Hq + hq) * T;
+        const double inv = 1.0 / sqrt((double)D);
+        double mx = sr[0] * inv;
+        for (int64_t t = 1; t < T; ++t)
+            if (sr[t] * inv > mx)
+                mx = sr[t] * inv;
+        double z = 0.0;
+        for (int64_t t = 0; t < T; ++t)
+            z += exp(sr[t] * inv - mx);
+        double *o = out + (b * Hq + hq) * D;
+        for (int64_t d = 0; d < D; ++d)
+            o[d] = 0.0;
+        for (int64_t t = 0; t < T; ++t) {
+            const double w = exp(sr[t] * inv - mx) / z * vscale[(b * T + t) * H + h];
+            const int8_t *vc = vcodes + ((b * T + t) * H + h) * D;
+            for (int64_t d = 0; d < D; ++d)
+                o[d] += w * (double)vc[d];
+        }
+    }
+    return 0;
+}
+
 int qo_max_threads(void)
 {
 #ifdef _OPENMP
