@@ -47,7 +47,7 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--cpu-rows", type=int, default=2048, help="token rows of the CPU-baseline sample")
     p.add_argument("--case", choices=["gemm", "gemm_group", "gemm8", "gemm8_full", "gemm_asym", "rotate",
-                                      "rotate_asym", "block", "kvquant", "kvscores"],
+                                      "rotate_asym", "block", "kvquant", "kvscores", "kvattend"],
                    default=None, help="time one kernel on a capture-sized workload (for ncu), not the step")
     return p.parse_args()
 
@@ -68,6 +68,7 @@ KERNEL_SOURCES = {
     "fwht_quant_kernel": ["rotate_quant.cuh", "tc_ptx.cuh", "common.cuh"],
     "kv_quant_tma_kernel_keys": ["kv_quant.cuh", "rotate_quant.cuh", "tc_ptx.cuh", "common.cuh"],
     "kv_scores_kernel": ["kv_scores.cuh", "common.cuh"],
+    "kv_attend_kernel": ["kv_attend.cuh", "common.cuh"],
 }
 
 
@@ -153,6 +154,11 @@ def bytes_kv_quant(B, T, H, D):
 
 def bytes_kv_scores(B, T, H, D, Hq):
     return B * T * H * (D // 2 + 2) + B * Hq * D * 2 + B * Hq * T * 4
+
+
+def bytes_kv_attend(B, T, H, D, Hq):
+    """fp32 scores in, packed value codes + fp16 value scales in, fp32 outputs out."""
+    return B * Hq * T * 4 + B * T * H * (D // 2 + 2) + B * Hq * D * 4
 
 
 # ---------------------------------------------------------------------------------------------
@@ -468,9 +474,14 @@ def run_case(args):
         if args.case == "kvquant":
             fn = lambda: q.quarot_kv_quant(k, v, s, kq, ks, vq, vs)
             work = bytes_kv_quant(B, T, H, D) / 1e9
-        else:
+        elif args.case == "kvscores":
             fn = lambda: q.quarot_kv_decode_scores(qh, s, kq, ks, scores)
             work = bytes_kv_scores(B, T, H, D, Hq) / 1e9
+        else:
+            q.quarot_kv_decode_scores(qh, s, kq, ks, scores)
+            o = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+            fn = lambda: q.quarot_kv_decode_attend(scores, vq, vs, o)
+            work = bytes_kv_attend(B, T, H, D, Hq) / 1e9
         unit = "GB/s"
     for _ in range(args.warmup):
         fn()

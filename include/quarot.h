@@ -342,6 +342,24 @@ quarot_status_t quarot_kv_decode_scores(const void *q_f16, int64_t B, int64_t Hq
                                         float *scores, quarot_stream_t stream);
 
 /*
+ * quarot_kv_decode_attend -- the rest of one decode step of attention over
+ * the INT4 value cache [QR-A: the KV cache in 4 bits; DQ-12: the attention
+ * output x value product on quantized values, softmax outputs unquantized]:
+ *
+ *   p[b,hq,t]   = softmax over t of scores[b,hq,t] / sqrt(D)
+ *   out[b,hq,d] = sum_t p[b,hq,t] * vs[b,t,h] * vcode[b,t,h,d],  h = hq / (Hq/Hkv)
+ *
+ * The value rows are not rotated (quarot_kv_quant), so no inverse rotation
+ * follows.  scores: fp32 [B, Hq, T] (e.g. from quarot_kv_decode_scores);
+ * vq [B, T, Hkv, D/2] packed value codes and vs_f16 [B, T, Hkv] fp16 value
+ * scales (from quarot_kv_quant); out: fp32 [B, Hq, D].
+ * Limits: D == 128; T >= 1; Hq / Hkv in {1, 2, 4, 8, 16}; B, Hkv <= 65535.
+ */
+quarot_status_t quarot_kv_decode_attend(const float *scores, int64_t B, int64_t Hq, const uint8_t *vq,
+                                        const void *vs_f16, int64_t T, int64_t Hkv, int64_t D, float *out,
+                                        quarot_stream_t stream);
+
+/*
  * quarot_get_device_status -- synchronizes the current device, then reports
  * (and clears) the library's device-side error word: QUAROT_ERR_DEVICE_TIMEOUT
  * if any kernel since the last call gave up a bounded wait (every wait inside

@@ -45,6 +45,7 @@ _SIGS = {
     "quarot_int4_linear_asym": ([_P, _P, _P, _P, _I64, _P, _P, _P, _P, _I64, _I64, _P, _P], _INT),
     "quarot_kv_quant": ([_P, _P, _I64, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P], _INT),
     "quarot_kv_decode_scores": ([_P, _I64, _I64, _P, _P, _P, _I64, _I64, _I64, _P, _P], _INT),
+    "quarot_kv_decode_attend": ([_P, _I64, _I64, _P, _P, _I64, _I64, _I64, _P, _P], _INT),
     "quarot_get_device_status": ([], _INT),
     "quarot_status_string": ([_INT], ctypes.c_char_p),
     "quarot_last_error": ([], ctypes.c_char_p),
@@ -303,6 +304,19 @@ def quarot_kv_decode_scores(q: torch.Tensor, signs: torch.Tensor, kq: torch.Tens
            lib.quarot_kv_decode_scores(_ptr(q), B, Hq, _ptr(signs), _ptr(kq), _ptr(ks), T, H, D, _ptr(scores),
                                        _stream(stream)))
     return scores
+
+
+def quarot_kv_decode_attend(scores: torch.Tensor, vq: torch.Tensor, vs: torch.Tensor,
+                            out: Optional[torch.Tensor] = None, stream=None):
+    """scores fp32 [B, Hq, T], vq [B, T, Hkv, 64], vs fp16 [B, T, Hkv] -> fp32 [B, Hq, 128]."""
+    B, Hq, T = scores.shape
+    Hkv = vq.shape[2]
+    if out is None:
+        out = torch.empty((B, Hq, 128), dtype=torch.float32, device=scores.device)
+    _check("quarot_kv_decode_attend",
+           lib.quarot_kv_decode_attend(_ptr(scores), B, Hq, _ptr(vq), _ptr(vs), T, Hkv, 128, _ptr(out),
+                                       _stream(stream)))
+    return out
 
 
 def quarot_get_device_status() -> int:

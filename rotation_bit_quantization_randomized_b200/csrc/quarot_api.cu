@@ -7,6 +7,7 @@
 #include "int4_gemm.cuh"
 #include "int4_gemm_pair.cuh"
 #include "int8_gemm_pair.cuh"
+#include "kv_attend.cuh"
 #include "kv_quant.cuh"
 #include "kv_scores.cuh"
 #include "rotate_quant.cuh"
@@ -921,6 +922,45 @@ quarot_status_t quarot_kv_decode_scores(const void *q_f16, int64_t B, int64_t Hq
     default: kv_scores_kernel<16><<<grid, kScoreThreads, 0, st>>>(qh, signs, k4, ksh, T, (int)Hkv, scores); break;
     }
     return after_launch("kv_scores_kernel launch");
+}
+
+quarot_status_t quarot_kv_decode_attend(const float *scores, int64_t B, int64_t Hq, const uint8_t *vq,
+                                        const void *vs_f16, int64_t T, int64_t Hkv, int64_t D, float *out,
+                                        quarot_stream_t stream)
+{
+    if (B < 0 || T <= 0 || Hkv <= 0 || Hq <= 0)
+        return fail(QUAROT_ERR_INVALID_ARG, "B must be >= 0; T, Hq, Hkv > 0");
+    if (D != 128)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "head dimension must be 128");
+    if (Hq % Hkv != 0)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "Hq must be a multiple of Hkv");
+    const int64_t G = Hq / Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "Hq / Hkv must be 1, 2, 4, 8 or 16");
+    if (Hkv > 65535 || B > 65535)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "B and Hkv must be <= 65535");
+    if (B == 0)
+        return QUAROT_OK;
+    if (!scores || !vq || !vs_f16 || !out)
+        return fail(QUAROT_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(scores) || !aligned16(vq) || !aligned16(vs_f16) || !aligned16(out))
+        return fail(QUAROT_ERR_MISALIGNED, "scores, codes, scales and output must be 16-byte aligned");
+    int dev;
+    DeviceInfo *info;
+    quarot_status_t s = current_device(dev, info);
+    if (s != QUAROT_OK)
+        return s;
+    dim3 grid((unsigned)Hkv, (unsigned)B);
+    cudaStream_t st = (cudaStream_t)stream;
+    const __half *vsh = static_cast<const __half *>(vs_f16);
+    switch (G) {
+    case 1: kv_attend_kernel<1><<<grid, kAttThreads, 0, st>>>(scores, vq, vsh, T, (int)Hkv, out); break;
+    case 2: kv_attend_kernel<2><<<grid, kAttThreads, 0, st>>>(scores, vq, vsh, T, (int)Hkv, out); break;
+    case 4: kv_attend_kernel<4><<<grid, kAttThreads, 0, st>>>(scores, vq, vsh, T, (int)Hkv, out); break;
+    case 8: kv_attend_kernel<8><<<grid, kAttThreads, 0, st>>>(scores, vq, vsh, T, (int)Hkv, out); break;
+    default: kv_attend_kernel<16><<<grid, kAttThreads, 0, st>>>(scores, vq, vsh, T, (int)Hkv, out); break;
+    }
+    return after_launch("kv_attend_kernel launch");
 }
 
 quarot_status_t quarot_get_device_status(void)

@@ -99,6 +99,14 @@ def test_kv_rejects(q):
     assert sc(A16, 1, 12, A16, A16, A16, 16, 8, 128, A16, None) == 2     # Hq % Hkv != 0
     assert sc(A16, 1, 64 * 8, A16, A16, A16, 16, 8, 128, A16, None) == 2  # group of 64
     assert sc(A16, 1, 64, A16, A16, A16, 0, 8, 128, None, None) == 0
+    at = q.lib.quarot_kv_decode_attend
+    assert at(A16, 1, 64, A16, A16, 16, 8, 64, A16, None) == 2       # D != 128
+    assert at(A16, 1, 12, A16, A16, 16, 8, 128, A16, None) == 2      # Hq % Hkv != 0
+    assert at(A16, 1, 24, A16, A16, 16, 8, 128, A16, None) == 2      # group of 3
+    assert at(A16, 1, 64, A16, A16, 0, 8, 128, A16, None) == 1       # no tokens
+    assert at(A16, 1, 64, A16, None, 16, 8, 128, A16, None) == 1
+    assert at(A16, 1, 64, MIS, A16, 16, 8, 128, A16, None) == 3
+    assert at(None, 0, 64, None, None, 16, 8, 128, None, None) == 0  # empty batch: no launch
 
 
 def test_binding_raises_on_error(q):
