@@ -950,16 +950,32 @@ quarot_status_t quarot_kv_decode_attend(const float *scores, int64_t B, int64_t 
     quarot_status_t s = current_device(dev, info);
     if (s != QUAROT_OK)
         return s;
-    dim3 grid((unsigned)Hkv, (unsigned)B);
-    cudaStream_t st = (cudaStream_t)stream;
+    // tokens split over a cluster of S CTAs, at least 128 tokens each
+    const int split = T >= 1024 ? 8 : T >= 512 ? 4 : T >= 256 ? 2 : 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)split, (unsigned)Hkv, (unsigned)B);
+    cfg.blockDim = dim3(kAttThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = (cudaStream_t)stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)split;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     const __half *vsh = static_cast<const __half *>(vs_f16);
+    const int hkv = (int)Hkv;
+    cudaError_t e;
     switch (G) {
-    case 1: kv_attend_kernel<1><<<grid, kAttThreads, 0, st>>>(scores, vq, vsh, T, (int)Hkv, out); break;
-    case 2: kv_attend_kernel<2><<<grid, kAttThreads, 0, st>>>(scores, vq, vsh, T, (int)Hkv, out); break;
-    case 4: kv_attend_kernel<4><<<grid, kAttThreads, 0, st>>>(scores, vq, vsh, T, (int)Hkv, out); break;
-    case 8: kv_attend_kernel<8><<<grid, kAttThreads, 0, st>>>(scores, vq, vsh, T, (int)Hkv, out); break;
-    default: kv_attend_kernel<16><<<grid, kAttThreads, 0, st>>>(scores, vq, vsh, T, (int)Hkv, out); break;
+    case 1: e = cudaLaunchKernelEx(&cfg, kv_attend_kernel<1>, scores, vq, vsh, T, hkv, out); break;
+    case 2: e = cudaLaunchKernelEx(&cfg, kv_attend_kernel<2>, scores, vq, vsh, T, hkv, out); break;
+    case 4: e = cudaLaunchKernelEx(&cfg, kv_attend_kernel<4>, scores, vq, vsh, T, hkv, out); break;
+    case 8: e = cudaLaunchKernelEx(&cfg, kv_attend_kernel<8>, scores, vq, vsh, T, hkv, out); break;
+    default: e = cudaLaunchKernelEx(&cfg, kv_attend_kernel<16>, scores, vq, vsh, T, hkv, out); break;
     }
+    if (e != cudaSuccess)
+        return cuda_fail(e, "kv_attend_kernel launch");
     return after_launch("kv_attend_kernel launch");
 }
 

@@ -64,7 +64,8 @@ def _values(rng, B, T, H):
 
 
 @pytest.mark.parametrize("B,T,H,G", [(1, 1, 8, 8), (1, 7, 8, 8), (2, 64, 8, 8), (2, 1000, 8, 8),
-                                      (1, 513, 2, 1), (2, 65, 4, 16), (1, 300, 3, 2), (1, 129, 2, 4)])
+                                      (1, 513, 2, 1), (2, 65, 4, 16), (1, 300, 3, 2), (1, 129, 2, 4),
+                                      (1, 1500, 2, 8), (1, 5000, 1, 16), (3, 257, 2, 8)])
 def test_attend_matches_oracle(q, B, T, H, G):
     rng = np.random.default_rng(7 * T + G)
     vq, vs = _values(rng, B, T, H)
@@ -97,6 +98,19 @@ def test_attend_dominant_score_and_uniform_scores(q):
     # KV head 1: all scores equal -> the plain mean of the value rows
     np.testing.assert_allclose(got[0, G:], np.repeat(rows[0, :, 1].mean(0)[None], G, 0),
                                rtol=0, atol=4 * (T + 32) * 2.0 ** -24 * np.abs(rows[0, :, 1]).max())
+
+
+@pytest.mark.parametrize("slope", [1.0, -1.0])
+def test_attend_running_maximum_across_chunks(q, slope):
+    """Scores that rise (or fall) along the tokens: with a rising ramp every
+    chunk of every token slice raises the running maximum, so the rescaling of
+    the partial sums is exercised at each step."""
+    rng = np.random.default_rng(11)
+    B, T, H, G = 1, 6000, 2, 8
+    vq, vs = _values(rng, B, T, H)
+    ramp = slope * np.linspace(0.0, 400.0, T)
+    scores = (ramp[None, None, :] + rng.standard_normal((B, H * G, T)) * 5).astype(np.float32)
+    _attend_check(q, scores, vq, vs)
 
 
 def test_attend_empty_batch_is_a_no_op(q):
