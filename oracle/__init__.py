@@ -36,6 +36,8 @@ def lib():
         I64 = ctypes.c_int64
         sigs = {
             "qo_sylvester": [I64, P],
+            "qo_paley": [ctypes.c_int, ctypes.c_int, P],
+            "qo_rotate_kron": [P, I64, I64, P, ctypes.c_int, ctypes.c_int, P],
             "qo_fwht": [P, I64],
             "qo_rotate": [P, I64, I64, P, I64, P],
             "qo_rotate_dense": [P, I64, I64, P, I64, P],
@@ -137,6 +139,33 @@ def rotate(x16, signs, had_block: int = 0, dense: bool = False) -> np.ndarray:
     fn = lib().qo_rotate_dense if dense else lib().qo_rotate
     _check(fn(_p(xb), M, K, _p(s), had_block, _p(out)), "rotate")
     return out
+
+
+def paley(p: int, e: int = 1) -> np.ndarray:
+    """Paley's first-construction Hadamard matrix of order p^e + 1 (p^e = 3 mod 4), int8 +-1."""
+    n = p ** e + 1
+    H = np.empty((n, n), np.int8)
+    _check(lib().qo_paley(p, e, _p(H)), "paley")
+    return H
+
+
+def rotate_kron(x16, signs, p: int = 7, e: int = 3) -> np.ndarray:
+    """x' = (x * diag(s)) * (H_m (x) H_n) / sqrt(K), m = p^e + 1 (Paley), n = K / m
+    (Sylvester).  The default factor is the one for K = 11008 = 344 * 32."""
+    xb = f16_bits(x16)
+    M, K = xb.shape
+    s = _c(signs, np.int8)
+    assert s.shape == (K,)
+    out = np.empty((M, K), np.float64)
+    _check(lib().qo_rotate_kron(_p(xb), M, K, _p(s), p, e, _p(out)), "rotate_kron")
+    return out
+
+
+def rotate_quant_kron(x16, signs, group: int = 0, p: int = 7, e: int = 3):
+    """The full-rotation activation step: Kronecker rotation, quantize, pack."""
+    xr = rotate_kron(x16, signs, p, e)
+    codes, sc = quantize(xr, group)
+    return pack(codes), sc, xr
 
 
 # --- quantizer -------------------------------------------------------------

@@ -649,6 +649,242 @@ int qo_kv_attend(const double *scores, int64_t B, int64_t Hq, int64_t H, int64_t
     return 0;
 }
 
+/* ------------------------------------------------------------------------ */
+/* Full rotation for sizes that are not a power of two: K = m * n with n a    */
+/* power of two and m = q + 1 the order of a Paley Hadamard matrix.           */
+/* (QuaRot summary, Elamur Research: the references name Sloane's library of  */
+/* Hadamard matrices as the source of the non-power-of-two factors.  That     */
+/* library is not available here; Paley's first construction gives a         */
+/* Hadamard matrix of every order q + 1 with q a prime power, q = 3 mod 4 --  */
+/* for K = 11008 = 344 * 32, q = 343 = 7^3.  Any Hadamard factor gives an     */
+/* orthogonal rotation with entries +-1/sqrt(K); this one is the reading.)    */
+/* ------------------------------------------------------------------------ */
+
+/* GF(p^e), e <= 3: element c0 + c1 x + c2 x^2 (c_i in Z_p) has index
+ * c0 + c1 p + c2 p^2.  The modulus is the first monic f(x) = x^e + f[e-1]
+ * x^(e-1) + ... + f[0] (in the order of the index of (f[0], .., f[e-1]))
+ * with no root in Z_p; for e <= 3 that is irreducibility. */
+typedef struct {
+    int p, e, q;
+    int f[3];
+} qo_gf;
+
+static int gf_digits(const qo_gf *F, int a, int *c)
+{
+    for (int i = 0; i < F->e; ++i) {
+        c[i] = a % F->p;
+        a /= F->p;
+    }
+    return 0;
+}
+
+static int gf_index(const qo_gf *F, const int *c)
+{
+    int a = 0;
+    for (int i = F->e - 1; i >= 0; --i)
+        a = a * F->p + c[i];
+    return a;
+}
+
+static int gf_sub(const qo_gf *F, int a, int b)
+{
+    int ca[3], cb[3], cd[3];
+    gf_digits(F, a, ca);
+    gf_digits(F, b, cb);
+    for (int i = 0; i < F->e; ++i)
+        cd[i] = ((ca[i] - cb[i]) % F->p + F->p) % F->p;
+    return gf_index(F, cd);
+}
+
+/* Product of polynomials, then x^k (k >= e) replaced by x^(k-e) * (-f(x) + x^e). */
+static int gf_mul(const qo_gf *F, int a, int b)
+{
+    int ca[3], cb[3];
+    long prod[5] = {0, 0, 0, 0, 0};
+    gf_digits(F, a, ca);
+    gf_digits(F, b, cb);
+    for (int i = 0; i < F->e; ++i)
+        for (int j = 0; j < F->e; ++j)
+            prod[i + j] += (long)ca[i] * cb[j];
+    for (int k = 2 * F->e - 2; k >= F->e; --k) {
+        long t = prod[k] % F->p;
+        prod[k] = 0;
+        for (int i = 0; i < F->e; ++i)
+            prod[k - F->e + i] -= t * F->f[i];
+    }
+    int c[3];
+    for (int i = 0; i < F->e; ++i)
+        c[i] = (int)(((prod[i] % F->p) + F->p) % F->p);
+    return gf_index(F, c);
+}
+
+/* Quadratic character: 0 at 0, +1 on nonzero squares, -1 otherwise, as
+ * a^((q-1)/2) (Euler's criterion; the power is 1 or -1 in the field). */
+static int gf_chi(const qo_gf *F, int a)
+{
+    if (a == 0)
+        return 0;
+    int r = 1, base = a, k = (F->q - 1) / 2;
+    while (k > 0) {
+        if (k & 1)
+            r = gf_mul(F, r, base);
+        base = gf_mul(F, base, base);
+        k >>= 1;
+    }
+    return r == 1 ? 1 : -1;
+}
+
+static int is_prime(int p)
+{
+    if (p < 2)
+        return 0;
+    for (int d = 2; d * d <= p; ++d)
+        if (p % d == 0)
+            return 0;
+    return 1;
+}
+
+static int gf_init(qo_gf *F, int p, int e)
+{
+    if (!is_prime(p) || e < 1 || e > 3)
+        return -1;
+    F->p = p;
+    F->e = e;
+    F->q = 1;
+    for (int i = 0; i < e; ++i)
+        F->q *= p;
+    F->f[0] = F->f[1] = F->f[2] = 0;
+    if (e == 1)
+        return 0;
+    int nf = 1;
+    for (int i = 0; i < e; ++i)
+        nf *= p;
+    for (int idx = 0; idx < nf; ++idx) {
+        int t = idx;
+        for (int i = 0; i < e; ++i) {
+            F->f[i] = t % p;
+            t /= p;
+        }
+        int has_root = 0;
+        for (int x = 0; x < p && !has_root; ++x) {
+            long v = 1;                       /* x^e */
+            for (int i = 0; i < e; ++i)
+                v = v * x % p;
+            long xp = 1;
+            for (int i = 0; i < e; ++i) {
+                v += (long)F->f[i] * xp;
+                xp = xp * x % p;
+            }
+            has_root = (v % p) == 0;
+        }
+        if (!has_root)
+            return 0;
+    }
+    return -1;
+}
+
+/*
+ * Paley's first construction, q = p^e = 3 mod 4, order n = q + 1:
+ *   Q[i][j] = chi(a_i - a_j)  over the field elements a_0 .. a_{q-1} (index order),
+ *   S = [[0, 1^T], [-1, Q]],  H = I + S.
+ * chi(-1) = -1 when q = 3 mod 4, so Q and S are skew-symmetric, Q Q^T = q I - J
+ * and Q J = 0, hence S S^T = q I and H H^T = (q + 1) I.
+ * Writes H row-major (n x n, +-1).  Returns 0, or -1 for an unsupported (p, e).
+ */
+int qo_paley(int p, int e, int8_t *H)
+{
+    qo_gf F;
+    if (gf_init(&F, p, e) != 0 || F.q % 4 != 3)
+        return -1;
+    const int n = F.q + 1;
+    int8_t *chi = (int8_t *)malloc((size_t)F.q);
+    if (!chi)
+        return -2;
+    for (int a = 0; a < F.q; ++a)
+        chi[a] = (int8_t)gf_chi(&F, a);
+    H[0] = 1;
+    for (int j = 1; j < n; ++j) {
+        H[j] = 1;
+        H[(int64_t)j * n] = -1;
+    }
+    for (int i = 1; i < n; ++i)
+        for (int j = 1; j < n; ++j)
+            H[(int64_t)i * n + j] = i == j ? 1 : chi[gf_sub(&F, i - 1, j - 1)];
+    free(chi);
+    return 0;
+}
+
+/*
+ * The full rotation for K = m * n, m = p^e + 1 (Paley factor), n = K / m a
+ * power of two (Sylvester factor):
+ *     x' = (x * diag(s)) * (H_m (x) H_n) / sqrt(K),
+ * with element index i = a * n + b and (A (x) B)[(a,b)][(a',b')] = A[a][a'] B[b][b'].
+ * The Kronecker product is applied through its two factors: with X the
+ * m x n matrix of x * s, X' = H_m^T X H_n / sqrt(K), both products written out.
+ */
+int qo_rotate_kron(const uint16_t *x16, int64_t M, int64_t K, const int8_t *signs, int p, int e,
+                   double *out)
+{
+    if (M < 0 || p < 2 || e < 1 || e > 3)
+        return -1;
+    int64_t q = 1;
+    for (int i = 0; i < e; ++i)
+        q *= p;
+    const int64_t m = q + 1;
+    if (K % m != 0 || !is_pow2(K / m))
+        return -1;
+    const int64_t n = K / m;
+    int8_t *Hm = (int8_t *)malloc((size_t)(m * m));
+    int8_t *Hn = (int8_t *)malloc((size_t)(n * n));
+    if (!Hm || !Hn) {
+        free(Hm);
+        free(Hn);
+        return -2;
+    }
+    if (qo_paley(p, e, Hm) != 0 || qo_sylvester(n, Hn) != 0) {
+        free(Hm);
+        free(Hn);
+        return -1;
+    }
+    const double inv = 1.0 / sqrt((double)K);
+    int err = 0;
+#pragma omp parallel for schedule(dynamic)
+    for (int64_t r = 0; r < M; ++r) {
+        double *X = (double *)malloc(sizeof(double) * (size_t)K);
+        double *T = (double *)malloc(sizeof(double) * (size_t)K);
+        if (!X || !T) {
+            free(X);
+            free(T);
+#pragma omp atomic write
+            err = -2;
+            continue;
+        }
+        for (int64_t i = 0; i < K; ++i)
+            X[i] = qo_f16_to_f64(x16[r * K + i]) * (double)signs[i];
+        /* T = H_m^T X: T[a'][b] = sum_a H_m[a][a'] X[a][b] */
+        for (int64_t a2 = 0; a2 < m; ++a2)
+            for (int64_t b = 0; b < n; ++b) {
+                double acc = 0.0;
+                for (int64_t a = 0; a < m; ++a)
+                    acc += (double)Hm[a * m + a2] * X[a * n + b];
+                T[a2 * n + b] = acc;
+            }
+        /* X' = T H_n / sqrt(K): X'[a'][b'] = sum_b T[a'][b] H_n[b][b'] */
+        for (int64_t a2 = 0; a2 < m; ++a2)
+            for (int64_t b2 = 0; b2 < n; ++b2) {
+                double acc = 0.0;
+                for (int64_t b = 0; b < n; ++b)
+                    acc += T[a2 * n + b] * (double)Hn[b * n + b2];
+                out[r * K + a2 * n + b2] = acc * inv;
+            }
+        free(X);
+        free(T);
+    }
+    free(Hm);
+    free(Hn);
+    return err;
+}
+
 int qo_max_threads(void)
 {
 #ifdef _OPENMP
