@@ -47,7 +47,8 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--cpu-rows", type=int, default=2048, help="token rows of the CPU-baseline sample")
     p.add_argument("--case", choices=["gemm", "gemm_group", "gemm8", "gemm8_full", "gemm_asym", "rotate",
-                                      "rotate_asym", "block", "kvquant", "kvscores", "kvattend"],
+                                      "rotate_asym", "block", "kron", "kron_tok", "kvquant", "kvscores",
+                                      "kvattend"],
                    default=None, help="time one kernel on a capture-sized workload (for ncu), not the step")
     return p.parse_args()
 
@@ -69,6 +70,7 @@ KERNEL_SOURCES = {
     "kv_quant_tma_kernel_keys": ["kv_quant.cuh", "rotate_quant.cuh", "tc_ptx.cuh", "common.cuh"],
     "kv_scores_kernel": ["kv_scores.cuh", "common.cuh"],
     "kv_attend_kernel": ["kv_attend.cuh", "common.cuh"],
+    "kron_quant_kernel": ["kron_quant.cuh", "int4_gemm.cuh", "rotate_quant.cuh", "tc_ptx.cuh", "common.cuh"],
 }
 
 
@@ -452,6 +454,14 @@ def run_case(args):
         s = (torch.randint(0, 2, (K,), device=dev, generator=g) * 2 - 1).to(torch.int8)
         outs = q.quarot_rotate_quant_asym(x, s, 0.9)
         fn = lambda: q.quarot_rotate_quant_asym(x, s, 0.9, 0, *outs)
+        work, unit = bytes_rotate_quant(M, K) / 1e9, "GB/s"
+    elif args.case in ("kron", "kron_tok"):
+        M, K = 8192, 11008
+        group = 128 if args.case == "kron" else 0
+        x = torch.randn((M, K), device=dev, generator=g).half()
+        s = (torch.randint(0, 2, (K,), device=dev, generator=g) * 2 - 1).to(torch.int8)
+        qa, sa = q.quarot_rotate_quant_kron(x, s, group)
+        fn = lambda: q.quarot_rotate_quant_kron(x, s, group, qa, sa)
         work, unit = bytes_rotate_quant(M, K) / 1e9, "GB/s"
     elif args.case in ("rotate", "block"):
         M, K = (8192, 8192) if args.case == "rotate" else (8192, 11008)

@@ -14,6 +14,8 @@
  *         most fused into the weights, a few applied at inference; products
  *         in integers) and "Key points" (activations quantized on the fly with
  *         round-to-nearest; group-wise variant with group size 128).
+ *  [QR-R] The same summary, References, item 24: Sloane's library of Hadamard
+ *         matrices, the source of factors whose order is not a power of two.
  *  [QR-N] QuaRot news article (onlyaistuff.com): randomized Hadamard
  *         transformations and computational invariance.
  *  [DQ-1], [DQ-2], [DQ-12] DuQuant (chapterpal) Knowl 1 (Y = XW =
@@ -24,7 +26,8 @@
  * Conventions for every entry point:
  *  - All array pointers are DEVICE memory owned by the caller; the library
  *    allocates nothing (except where an entry point says otherwise) and keeps
- *    no state beyond a per-device cache of kernel attributes.
+ *    no state beyond a per-device cache of kernel attributes (and, once the
+ *    full Kronecker rotation has run on a device, its 288 KB Hadamard factor).
  *  - Every array pointer must be 16-byte aligned; arrays are dense row-major.
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *    default stream).  Argument errors are returned before any launch and
@@ -84,6 +87,37 @@ typedef void *quarot_stream_t;
 quarot_status_t quarot_rotate_quant(const void *x_f16, int64_t M, int64_t K,
                                     const int8_t *signs, int had_block, int group,
                                     uint8_t *q_packed, void *scales, quarot_stream_t stream);
+
+/*
+ * quarot_rotate_quant_kron -- the full (not block-diagonal) rotation for
+ * K = 11008, which is not a power of two, fused with INT4 RTN quantization
+ * and packing [QR-S Summary, Key points; QR-R; DQ-1]:
+ *
+ *   x' = (x * diag(signs)) * (H_344 (x) H_32) / sqrt(11008),  element i = 32 a + b,
+ *   (H_344 (x) H_32)[32a + b][32a' + b'] = H_344[a][a'] * H_32[b][b'],
+ *
+ * H_32 Sylvester-ordered; H_344 the library's Hadamard matrix of order 344
+ * (Paley's first construction over GF(7^3) = GF(7)[x]/(x^3 + 2), elements
+ * c0 + c1 x + c2 x^2 numbered c0 + 7 c1 + 49 c2; quarot_kron_factor returns
+ * it).  Quantization exactly as quarot_rotate_quant (group 0: fp32 scale per
+ * row; group 128: fp16 scale per 128 elements).  Every output element mixes
+ * all 11008 inputs, unlike had_block == 128.
+ *
+ * x_f16 [M, 11008] fp16; signs [11008] int8 (+1 / -1); q_packed [M, 5504]
+ * uint8 out; scales fp32 [M] (group 0) or fp16 [M, 86] (group 128) out.
+ * K must be 11008 (else QUAROT_ERR_UNSUPPORTED_SHAPE).  The first call on a
+ * device allocates and uploads the factor (288 KB, kept until exit).
+ */
+quarot_status_t quarot_rotate_quant_kron(const void *x_f16, int64_t M, int64_t K, const int8_t *signs,
+                                         int64_t group, uint8_t *q_packed, void *scales, quarot_stream_t stream);
+
+/*
+ * quarot_kron_factor -- writes the library's Hadamard factor of order m
+ * (only m == 344) to HOST memory h_out[m * m] (int8 +1 / -1, row-major), for
+ * rotating weights offline with the same matrix [QR-S Summary: the rotations
+ * are folded into the weights].  H H^T = m I.  Needs no device.
+ */
+quarot_status_t quarot_kron_factor(int64_t m, int8_t *h_out);
 
 /*
  * quarot_int4_linear -- INT4 x INT4 linear layer with int32 accumulation on

@@ -45,6 +45,8 @@ _SIGS = {
     "quarot_int4_linear_asym": ([_P, _P, _P, _P, _I64, _P, _P, _P, _P, _I64, _I64, _P, _P], _INT),
     "quarot_kv_quant": ([_P, _P, _I64, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P], _INT),
     "quarot_kv_decode_scores": ([_P, _I64, _I64, _P, _P, _P, _I64, _I64, _I64, _P, _P], _INT),
+    "quarot_rotate_quant_kron": ([_P, _I64, _I64, _P, _I64, _P, _P, _P], _INT),
+    "quarot_kron_factor": ([_I64, _P], _INT),
     "quarot_kv_decode_attend": ([_P, _I64, _I64, _P, _P, _I64, _I64, _I64, _P, _P], _INT),
     "quarot_get_device_status": ([], _INT),
     "quarot_status_string": ([_INT], ctypes.c_char_p),
@@ -304,6 +306,27 @@ def quarot_kv_decode_scores(q: torch.Tensor, signs: torch.Tensor, kq: torch.Tens
            lib.quarot_kv_decode_scores(_ptr(q), B, Hq, _ptr(signs), _ptr(kq), _ptr(ks), T, H, D, _ptr(scores),
                                        _stream(stream)))
     return scores
+
+
+def quarot_rotate_quant_kron(x: torch.Tensor, signs: torch.Tensor, group: int = 0,
+                             q: Optional[torch.Tensor] = None, scales: Optional[torch.Tensor] = None, stream=None):
+    """Full Kronecker rotation (K = 11008 = 344 * 32) + INT4 RTN + packing -> (q [M, K/2] uint8, scales)."""
+    M, K = x.shape
+    if q is None:
+        q = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((M,), dtype=torch.float32, device=x.device) if group == 0 else \
+            torch.empty((M, K // 128), dtype=torch.float16, device=x.device)
+    _check("quarot_rotate_quant_kron",
+           lib.quarot_rotate_quant_kron(_ptr(x), M, K, _ptr(signs), group, _ptr(q), _ptr(scales), _stream(stream)))
+    return q, scales
+
+
+def quarot_kron_factor(m: int = 344):
+    """The library's Hadamard factor of order m (host int8 tensor [m, m])."""
+    h = torch.empty((m, m), dtype=torch.int8)
+    _check("quarot_kron_factor", lib.quarot_kron_factor(m, h.data_ptr()))
+    return h
 
 
 def quarot_kv_decode_attend(scores: torch.Tensor, vq: torch.Tensor, vs: torch.Tensor,

@@ -7,6 +7,7 @@
 #include "int4_gemm.cuh"
 #include "int4_gemm_pair.cuh"
 #include "int8_gemm_pair.cuh"
+#include "kron_quant.cuh"
 #include "kv_attend.cuh"
 #include "kv_quant.cuh"
 #include "kv_scores.cuh"
@@ -18,6 +19,7 @@
 #include <cstdio>
 #include <mutex>
 #include <string>
+#include <vector>
 
 using namespace quarot;
 
@@ -549,6 +551,132 @@ quarot_status_t noalloc_scratch_address(int dev, void *&addr)
     return QUAROT_OK;
 }
 
+// ----------------------------------------------------------------- full Kronecker rotation
+// The Hadamard factor of order 344 by Paley's first construction: q = 343 =
+// 7^3 = 3 mod 4, field GF(7)[x] / (x^3 + 2) (x^3 + 2 has no root in GF(7),
+// whose cubes are 0, 1 and 6, so it is irreducible), element
+// c0 + c1 x + c2 x^2 numbered c0 + 7 c1 + 49 c2.  With chi the quadratic
+// character (found here by squaring every nonzero element):
+//   H[0][j] = 1, H[i][0] = -1 (i > 0), H[i][i] = 1,
+//   H[i][j] = chi(e_{i-1} - e_{j-1}) otherwise,
+// so H H^T = 344 I.
+void paley344(int8_t *H)
+{
+    constexpr int p = 7, q = 343, n = 344;
+    auto digits = [](int a, int (&c)[3]) {
+        c[0] = a % p;
+        c[1] = (a / p) % p;
+        c[2] = a / (p * p);
+    };
+    auto mul = [&](int a, int b) {
+        int A[3], B[3];
+        digits(a, A);
+        digits(b, B);
+        int P[5] = {0, 0, 0, 0, 0};
+        for (int i = 0; i < 3; ++i)
+            for (int j = 0; j < 3; ++j)
+                P[i + j] += A[i] * B[j];
+        P[1] += 5 * P[4];                  // x^4 = x * x^3 = 5 x
+        P[0] += 5 * P[3];                  // x^3 = -2 = 5
+        return P[0] % p + p * (P[1] % p) + p * p * (P[2] % p);
+    };
+    std::vector<int8_t> square(q, 0);
+    for (int y = 1; y < q; ++y)
+        square[mul(y, y)] = 1;
+    auto chi_diff = [&](int a, int b) {
+        int A[3], B[3];
+        digits(a, A);
+        digits(b, B);
+        const int d = (A[0] - B[0] + p) % p + p * ((A[1] - B[1] + p) % p) + p * p * ((A[2] - B[2] + p) % p);
+        return d == 0 ? 0 : (square[d] ? 1 : -1);
+    };
+    for (int j = 0; j < n; ++j)
+        H[j] = 1;
+    for (int i = 1; i < n; ++i) {
+        H[(size_t)i * n] = -1;
+        for (int j = 1; j < n; ++j)
+            H[(size_t)i * n + j] = (int8_t)(i == j ? 1 : chi_diff(i - 1, j - 1));
+    }
+}
+
+// H^T as fp16, zero-padded to 384 x 384 (the MMA operand), once per device.
+std::mutex g_kron_mutex;
+void *g_kron_factor[kMaxDevices] = {};
+
+quarot_status_t kron_factor_device(int dev, const void *&ptr)
+{
+    std::lock_guard<std::mutex> lk(g_kron_mutex);
+    if (!g_kron_factor[dev]) {
+        std::vector<int8_t> H((size_t)kKronM * kKronM);
+        paley344(H.data());
+        std::vector<uint16_t> Ht((size_t)kKronAPad * kKronAPad, 0);
+        for (int ap = 0; ap < kKronM; ++ap)
+            for (int a = 0; a < kKronM; ++a)
+                Ht[(size_t)ap * kKronAPad + a] = H[(size_t)a * kKronM + ap] > 0 ? 0x3C00 : 0xBC00;
+        void *d = nullptr;
+        cudaError_t e = cudaMalloc(&d, Ht.size() * 2);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cudaMalloc (Hadamard factor)");
+        e = cudaMemcpy(d, Ht.data(), Ht.size() * 2, cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) {
+            cudaFree(d);
+            return cuda_fail(e, "cudaMemcpy (Hadamard factor)");
+        }
+        g_kron_factor[dev] = d;
+    }
+    ptr = g_kron_factor[dev];
+    return QUAROT_OK;
+}
+
+quarot_status_t kron_launch(const void *x, int64_t M, const int8_t *signs, int group, uint8_t *q, void *scales,
+                            cudaStream_t st)
+{
+    int dev;
+    DeviceInfo *info;
+    quarot_status_t s = current_device(dev, info);
+    if (s != QUAROT_OK)
+        return s;
+    const void *ht;
+    s = kron_factor_device(dev, ht);
+    if (s != QUAROT_OK)
+        return s;
+    EncodeTiledFn fn;
+    s = encode_tiled_fn(fn);
+    if (s != QUAROT_OK)
+        return s;
+    CUtensorMap map;
+    const cuuint64_t dims[2] = {(cuuint64_t)kKronAPad, (cuuint64_t)kKronAPad};
+    const cuuint64_t strides[1] = {(cuuint64_t)kKronAPad * 2};
+    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(ht), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(QUAROT_ERR_CUDA, "cuTensorMapEncodeTiled failed (code " + std::to_string((int)r) + ")");
+    const size_t smem = KronSmem::kBytes;
+    const float scale_mul = (float)(1.0 / (7.0 * std::sqrt((double)kKronK)));
+    const float sqrt_n = (float)std::sqrt((double)kKronK);
+    const int64_t tiles = (M + kKronRows - 1) / kKronRows;
+    int per_sm = 0;
+    if (group == 0) {
+        s = kernel_occupancy(kron_quant_kernel<0>, dev, kKronThreads, smem, per_sm);
+        if (s != QUAROT_OK)
+            return s;
+        const int grid = (int)std::min<int64_t>(tiles, (int64_t)info->sm_count * per_sm);
+        kron_quant_kernel<0><<<grid, kKronThreads, smem, st>>>(map, static_cast<const __half *>(x), M, signs, q,
+                                                               scales, scale_mul, sqrt_n);
+    } else {
+        s = kernel_occupancy(kron_quant_kernel<128>, dev, kKronThreads, smem, per_sm);
+        if (s != QUAROT_OK)
+            return s;
+        const int grid = (int)std::min<int64_t>(tiles, (int64_t)info->sm_count * per_sm);
+        kron_quant_kernel<128><<<grid, kKronThreads, smem, st>>>(map, static_cast<const __half *>(x), M, signs, q,
+                                                                 scales, scale_mul, sqrt_n);
+    }
+    return after_launch("kron_quant_kernel launch");
+}
+
 }  // namespace
 
 // Tensor map of an fp16 [rows, 128] matrix (KV rows of one head) read in
@@ -602,6 +730,34 @@ quarot_status_t quarot_rotate_quant(const void *x_f16, int64_t M, int64_t K, con
     if (s != QUAROT_OK || M == 0)
         return s;
     return rotate_quant_launch(x_f16, M, K, signs, had_block, group, q_packed, scales, (cudaStream_t)stream);
+}
+
+quarot_status_t quarot_rotate_quant_kron(const void *x_f16, int64_t M, int64_t K, const int8_t *signs,
+                                         int64_t group, uint8_t *q_packed, void *scales, quarot_stream_t stream)
+{
+    if (M < 0)
+        return fail(QUAROT_ERR_INVALID_ARG, "M must be >= 0");
+    if (group != 0 && group != 128)
+        return fail(QUAROT_ERR_INVALID_ARG, "group must be 0 or 128");
+    if (K != kKronK)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "the full Kronecker rotation supports K = 11008 = 344 * 32");
+    if (M == 0)
+        return QUAROT_OK;
+    if (!x_f16 || !signs || !q_packed || !scales)
+        return fail(QUAROT_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(x_f16) || !aligned16(signs) || !aligned16(q_packed) || !aligned16(scales))
+        return fail(QUAROT_ERR_MISALIGNED, "x, signs, codes and scales must be 16-byte aligned");
+    return kron_launch(x_f16, M, signs, (int)group, q_packed, scales, (cudaStream_t)stream);
+}
+
+quarot_status_t quarot_kron_factor(int64_t m, int8_t *h_out)
+{
+    if (m != kKronM)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "the library's non-power-of-two factor has order 344");
+    if (!h_out)
+        return fail(QUAROT_ERR_INVALID_ARG, "null pointer");
+    paley344(h_out);
+    return QUAROT_OK;
 }
 
 quarot_status_t quarot_int4_linear(const uint8_t *qa, const void *s_a, int64_t M, const uint8_t *qw,

@@ -109,6 +109,23 @@ def test_kv_rejects(q):
     assert at(None, 0, 64, None, None, 16, 8, 128, None, None) == 0  # empty batch: no launch
 
 
+def test_kron_entry_point_rejects_and_factor_matches_oracle(q):
+    import numpy as np
+    import oracle
+    kr = q.lib.quarot_rotate_quant_kron
+    assert kr(A16, 4, 11008 - 128, A16, 0, A16, A16, None) == 2     # only K = 11008
+    assert kr(A16, 4, 11008, A16, 64, A16, A16, None) == 1          # group 0 or 128
+    assert kr(A16, -1, 11008, A16, 0, A16, A16, None) == 1
+    assert kr(A16, 4, 11008, None, 0, A16, A16, None) == 1
+    assert kr(MIS, 4, 11008, A16, 0, A16, A16, None) == 3
+    assert kr(None, 0, 11008, None, 0, None, None, None) == 0       # empty: no launch
+    assert q.lib.quarot_kron_factor(172, A16) == 2
+    # the library's factor (squares enumerated) equals the oracle's (Euler's
+    # criterion): two independent routes to the same Paley matrix
+    h = q.quarot_kron_factor(344).numpy()
+    np.testing.assert_array_equal(h, oracle.paley(7, 3))
+
+
 def test_binding_raises_on_error(q):
     import torch
     x = torch.zeros((4, 384), dtype=torch.float16)
