@@ -21,7 +21,7 @@
 //     from global memory (L2-resident) by TMA in 128 x 64 blocks;
 // B = the tile's (x * s)^T, 128 rows (r, b) x 352 reduction columns a, kept
 //     as six 64-column slots: the copy engine brings each 64-column slice of
-//     the 4 rows (4 x 4 KB, contiguous in x) into a staging ring; four
+//     the 4 rows (4 x 4 KB, contiguous in x) into a staging ring; eight
 //     transposer warps flip the sign bits, transpose 8 x 8 fp16 blocks in
 //     registers and store them in the swizzled K-major layout;
 // the MMAs run a'-tile by a'-tile (t outer, k inner), so accumulator D_t is
@@ -37,8 +37,9 @@
 //    over the 128 lanes and 3 tiles), a second pass quantizes;
 //  * group 128: a group is 4 consecutive a' (4 adjacent lanes): the scale
 //    comes from a 2-step shuffle maximum.
-// Warp roles: 0-7 epilogue, 8-11 transposers, 12 x loader, 13 factor loader,
-// 14 MMA issuer.  Every wait is bounded (an abort flag stops all roles).
+// Warp roles: 0-7 epilogue, 8-15 transposers (two groups taking alternate
+// 64-column slices; signs flipped through a 256-entry mask table), 16 x
+// loader, 17 factor loader, 18 MMA issuer.  Every wait is bounded (an abort flag stops all roles).
 #pragma once
 
 #include <cuda.h>
@@ -57,11 +58,11 @@ constexpr int kKronRows = 4;                   // tokens per tile
 constexpr int kKronKB = 6;                     // 64-column blocks of the reduction (352 used)
 constexpr int kKronAT = 3;                     // 128-row blocks of a' (384)
 constexpr int kKronBlock = 16384;              // bytes of one 128 x 64 fp16 block
-constexpr int kKronAStages = 5, kKronXStages = 2;
+constexpr int kKronAStages = 4, kKronXStages = 3;
 constexpr int kKronEpiWarps = 8;
-constexpr int kKronTrWarp0 = 8;                // transposers: warps 8-11
-constexpr int kKronXWarp = 12, kKronAWarp = 13, kKronMmaWarp = 14;
-constexpr int kKronThreads = 15 * 32;
+constexpr int kKronTrWarp0 = 8;                // transposers: warps 8-15, two groups of 4
+constexpr int kKronXWarp = 16, kKronAWarp = 17, kKronMmaWarp = 18;
+constexpr int kKronThreads = 19 * 32;
 
 struct KronSmem {
     static constexpr int kAOff = 0;
@@ -70,7 +71,11 @@ struct KronSmem {
     static constexpr int kBarOff = kXOff + kKronXStages * kKronBlock;
     static constexpr int kNumBars = 2 * kKronXStages + 2 * kKronKB + 2 * kKronAStages + 2 * kKronAT + 1;
     static constexpr int kMiscOff = kBarOff + 8 * kNumBars;
-    static constexpr int kBytes = kMiscOff + 16 + 4 * kKronEpiWarps * 2 + 1024;   // slot/flag, reduction, alignment
+    static constexpr int kLutOff = (kMiscOff + 16 + 4 * kKronEpiWarps * 2 + 15) / 16 * 16;   // after slot/flag, reduction
+    static constexpr int kSignOff = kLutOff + 256 * 16;                         // 256 sign-mask patterns
+    static constexpr int kBytes = kSignOff + 4 * kKronM + 1024;                 // sign bytes [4][344], alignment
+    static_assert(kLutOff % 16 == 0 && kSignOff % 16 == 0 && kMiscOff % 8 == 0, "shared-memory alignment");
+    static_assert(kBytes <= 232448, "shared memory per block");
 };
 
 // Instruction descriptor for kind::f16: fp32 accumulator, fp16 A and B, both K-major.
@@ -137,14 +142,15 @@ __device__ __forceinline__ uint4 quant_pack32(const float (&v)[32], float r)
     return make_uint4(pk[0], pk[1], pk[2], pk[3]);
 }
 
-// Sign-bit masks of 8 fp16 values from 8 sign bytes (+1 / -1): word w gets
-// bit 15 from byte 2w and bit 31 from byte 2w + 1.
-__device__ __forceinline__ void sign_masks8(uint2 sb, uint32_t (&m)[4])
+// XOR masks that flip the signs of 8 fp16 values (4 words) whose sign bits
+// are the 8 bits of v: word w gets bit 15 from bit 2w and bit 31 from bit 2w + 1.
+__device__ __forceinline__ uint4 sign_mask_pattern(uint32_t v)
 {
-    m[0] = __byte_perm(sb.x, 0u, 0x1404) & 0x80008000u;
-    m[1] = __byte_perm(sb.x, 0u, 0x3424) & 0x80008000u;
-    m[2] = __byte_perm(sb.y, 0u, 0x1404) & 0x80008000u;
-    m[3] = __byte_perm(sb.y, 0u, 0x3424) & 0x80008000u;
+    uint32_t m[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w)
+        m[w] = (((v >> (2 * w)) & 1u) << 15) | (((v >> (2 * w + 1)) & 1u) << 31);
+    return make_uint4(m[0], m[1], m[2], m[3]);
 }
 
 template <int GROUP>
@@ -202,6 +208,25 @@ kron_quant_kernel(const __grid_constant__ CUtensorMap tma_h,     // H^T, fp16 [3
     if (warp == kKronMmaWarp) {
         tmem_alloc(smem_u32(tmem_slot), 512);
         tmem_relinquish();
+    }
+    // sign bits of x as bytes sbyte[j][a] (bit bb = s[32 a + 8 j + bb] < 0) and
+    // the 256 mask patterns, so that the transposers flip signs from shared memory
+    {
+        uint4 *lut = reinterpret_cast<uint4 *>(smem + S::kLutOff);
+        uint8_t *sbyte = smem + S::kSignOff;
+        for (int v = threadIdx.x; v < 256; v += kKronThreads)
+            lut[v] = sign_mask_pattern((uint32_t)v);
+        for (int i = threadIdx.x; i < 4 * kKronM; i += kKronThreads) {
+            const int j = i / kKronM, a = i - j * kKronM;
+            const uint2 sb = __ldg(reinterpret_cast<const uint2 *>(signs + a * kKronN + 8 * j));
+            uint32_t bits = 0;
+#pragma unroll
+            for (int bb = 0; bb < 8; ++bb) {
+                const uint32_t byte = ((bb < 4 ? sb.x : sb.y) >> (8 * (bb & 3))) & 0xFFu;
+                bits |= ((byte >> 7) & 1u) << bb;
+            }
+            sbyte[i] = (uint8_t)bits;
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -311,14 +336,18 @@ kron_quant_kernel(const __grid_constant__ CUtensorMap tma_h,     // H^T, fp16 [3
         __syncwarp();
     } else if (warp >= kKronTrWarp0) {
         // ------------------------------------------------------------ transposers
-        // thread u: token r = u / 32 (its warp), 8 x 8 block (c, j): columns
-        // a = 64 kb + 8 c + i (i = 0..7), b = 8 j .. 8 j + 7
-        const int u = threadIdx.x - 32 * kKronTrWarp0;
+        // group g = 0 / 1 takes the k-blocks kb = g, g + 2, g + 4 of every tile.
+        // thread u of a group: token r = u / 32 (its warp), 8 x 8 block (c, j):
+        // columns a = 64 kb + 8 c + i (i = 0..7), b = 8 j .. 8 j + 7
+        const int tg = (warp - kKronTrWarp0) >> 2;
+        const int u = threadIdx.x - 32 * kKronTrWarp0 - 128 * tg;
         const int r = u >> 5, c = (u >> 2) & 7, j = u & 3;
+        const uint4 *lut = reinterpret_cast<const uint4 *>(smem + S::kLutOff);
+        const uint8_t *sbyte = smem + S::kSignOff + j * kKronM;
         bool ok = true;
-        int step = 0;
         for (int lt = 0; lt < my_tiles && ok; ++lt) {
-            for (int kb = 0; kb < kKronKB; ++kb, ++step) {
+            for (int kb = tg; kb < kKronKB; kb += 2) {
+                const int step = lt * kKronKB + kb;
                 const int xs = step % kKronXStages;
                 ok = gemm_wait_warp(bar_xfull + 8 * xs, (uint32_t)(step / kKronXStages) & 1, abort_flag) &&
                      gemm_wait_warp(bar_bempty + 8 * kb, ((uint32_t)lt & 1) ^ 1, abort_flag);
@@ -328,17 +357,16 @@ kron_quant_kernel(const __grid_constant__ CUtensorMap tma_h,     // H^T, fp16 [3
                 uint8_t *bdst = smem + S::kBOff + kb * kKronBlock;
                 if (a0 < kKronM) {
                     const uint8_t *src = smem + S::kXOff + xs * kKronBlock + r * 4096 + (8 * c) * 64 + 16 * j;
+                    const uint2 sw = *reinterpret_cast<const uint2 *>(sbyte + a0);     // sign bytes of a0 .. a0 + 7
                     uint4 in[8];
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         in[i] = *reinterpret_cast<const uint4 *>(src + 64 * i);
-                        const uint2 sb = __ldg(reinterpret_cast<const uint2 *>(signs + (a0 + i) * kKronN + 8 * j));
-                        uint32_t m[4];
-                        sign_masks8(sb, m);
-                        in[i].x ^= m[0];
-                        in[i].y ^= m[1];
-                        in[i].z ^= m[2];
-                        in[i].w ^= m[3];
+                        const uint4 m = lut[((i < 4 ? sw.x : sw.y) >> (8 * (i & 3))) & 0xFFu];
+                        in[i].x ^= m.x;
+                        in[i].y ^= m.y;
+                        in[i].z ^= m.z;
+                        in[i].w ^= m.w;
                     }
                     // out[bb] = the 8 values of column b = 8 j + bb, a = a0 .. a0 + 7
 #pragma unroll
