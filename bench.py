@@ -226,6 +226,23 @@ def run_reference(args, rank):
 
 
 # ---------------------------------------------------------------------------------------------
+# rank coordination (replicas only: the only collectives are the barrier and these reductions)
+
+def max_over_ranks(x, dist, device=None):
+    """The largest x over the ranks of the process group (x itself without one):
+    every timed quantity is reported as its slowest rank's."""
+    if dist is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(work_per_rank, world, seconds):
+    """Whole-job throughput under weak scaling: every rank does the same work."""
+    return work_per_rank * world / seconds
+
 
 def run_ours(args, rank, world, local_rank, dist):
     import torch
@@ -306,15 +323,11 @@ def run_ours(args, rank, world, local_rank, dist):
     per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(args.steps)])
     k_ms = per.mean(axis=0)
 
-    if dist is not None:
-        import torch.distributed as tdist
-        t = torch.tensor([total_ms], device=dev)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist, dev)
 
     ms_step = total_ms / args.steps
     ops = 2.0 * M * N * K
-    value = ops * world / (ms_step * 1e-3) / 1e12
+    value = job_rate(ops, world, ms_step * 1e-3) / 1e12
     pk = peaks()
     int8_sust = 2.0 * pk["bf16_sust"]
     gemm_tops = ops / (k_ms[1] * 1e-3) / 1e12
@@ -356,12 +369,8 @@ def run_ours(args, rank, world, local_rank, dist):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-    if dist is not None:
-        import torch.distributed as tdist
-        t = torch.tensor([e2e_ms], device=dev)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = ops * world / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
+    e2e_value = job_rate(ops, world, e2e_ms * 1e-3) / 1e12
 
     cpu = None
     if rank == 0 and world == 1:
