@@ -48,7 +48,7 @@ def parse():
     p.add_argument("--cpu-rows", type=int, default=2048, help="token rows of the CPU-baseline sample")
     p.add_argument("--case", choices=["gemm", "gemm_group", "gemm8", "gemm8_full", "gemm_asym", "rotate",
                                       "rotate_asym", "block", "kron", "kron_tok", "kvquant", "kvscores",
-                                      "kvattend"],
+                                      "kvattend", "kvattend_b64"],
                    default=None, help="time one kernel on a capture-sized workload (for ncu), not the step")
     return p.parse_args()
 
@@ -483,7 +483,7 @@ def run_case(args):
         fn = lambda: q.quarot_rotate_quant(x, s, hb, group, qa, sa)
         work, unit = bytes_rotate_quant(M, K) / 1e9, "GB/s"
     else:
-        B, T, H, D, Hq = 16, 2048, 8, 128, 64
+        B, T, H, D, Hq = (64 if args.case == "kvattend_b64" else 16), 2048, 8, 128, 64
         k = torch.randn((B, T, H, D), device=dev, generator=g).half()
         v = torch.randn((B, T, H, D), device=dev, generator=g).half()
         qh = torch.randn((B, Hq, D), device=dev, generator=g).half()

@@ -8,8 +8,8 @@
 //
 // The value rows were stored unrotated, so no inverse rotation follows.
 //
-// A cluster of S CTAs (S = 1, 2, 4 or 8, by T) covers one (batch, kv-head)
-// pair; CTA r takes the r-th slice of the tokens, for all G query heads that
+// A cluster of S CTAs (S = 1, 2, 4 or 8, chosen on the host from T and from
+// how many clusters can be resident at once) covers one (batch, kv-head) pair; CTA r takes the r-th slice of the tokens, for all G query heads that
 // share the head, so each value nibble is read once and used G times.  Within
 // its slice a CTA walks chunks of 256 tokens with the running-maximum form of
 // the softmax (per head: maximum m, sum of exponentials l, and the

@@ -677,6 +677,47 @@ quarot_status_t kron_launch(const void *x, int64_t M, const int8_t *signs, int g
     return after_launch("kron_quant_kernel launch");
 }
 
+// Clusters of `split` attention CTAs (G query heads per KV head) that can be
+// resident at once on the device, queried once per (device, G, split).
+quarot_status_t attend_resident_clusters(int G, int split, int dev, int &fit)
+{
+    static int cache[kMaxDevices][5][4];
+    static bool known[kMaxDevices][5][4];
+    const int gi = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : G == 8 ? 3 : 4;
+    const int si = split == 1 ? 0 : split == 2 ? 1 : split == 4 ? 2 : 3;
+    {
+        std::lock_guard<std::mutex> lk(g_mutex);
+        if (known[dev][gi][si]) {
+            fit = cache[dev][gi][si];
+            return QUAROT_OK;
+        }
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)split, 1, 1);
+    cfg.blockDim = dim3(kAttThreads);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)split;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
+    switch (G) {
+    case 1: e = cudaOccupancyMaxActiveClusters(&fit, kv_attend_kernel<1>, &cfg); break;
+    case 2: e = cudaOccupancyMaxActiveClusters(&fit, kv_attend_kernel<2>, &cfg); break;
+    case 4: e = cudaOccupancyMaxActiveClusters(&fit, kv_attend_kernel<4>, &cfg); break;
+    case 8: e = cudaOccupancyMaxActiveClusters(&fit, kv_attend_kernel<8>, &cfg); break;
+    default: e = cudaOccupancyMaxActiveClusters(&fit, kv_attend_kernel<16>, &cfg); break;
+    }
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaOccupancyMaxActiveClusters");
+    std::lock_guard<std::mutex> lk(g_mutex);
+    cache[dev][gi][si] = fit;
+    known[dev][gi][si] = true;
+    return QUAROT_OK;
+}
+
 }  // namespace
 
 // Tensor map of an fp16 [rows, 128] matrix (KV rows of one head) read in
@@ -1106,8 +1147,28 @@ quarot_status_t quarot_kv_decode_attend(const float *scores, int64_t B, int64_t 
     quarot_status_t s = current_device(dev, info);
     if (s != QUAROT_OK)
         return s;
-    // tokens split over a cluster of S CTAs, at least 128 tokens each
-    const int split = T >= 1024 ? 8 : T >= 512 ? 4 : T >= 256 ? 2 : 1;
+    // tokens split over a cluster of S CTAs, at least 128 tokens each: the S
+    // whose B * Hkv * S CTAs fill the resident slots best (CTAs / (waves x
+    // resident CTAs)); on a tie the one with fewer waves (no tail wave that
+    // runs on a few SMs only)
+    const int smax = T >= 1024 ? 8 : T >= 512 ? 4 : T >= 256 ? 2 : 1;
+    int split = smax;
+    double best_eff = -1.0;
+    int64_t best_waves = 0;
+    for (int sp = smax; sp >= 1; sp /= 2) {
+        int fit = 0;
+        s = attend_resident_clusters((int)G, sp, dev, fit);
+        if (s != QUAROT_OK)
+            return s;
+        const int64_t clusters = B * Hkv;
+        const int64_t waves = fit > 0 ? (clusters + fit - 1) / fit : clusters;
+        const double eff = fit > 0 ? (double)clusters / ((double)waves * fit) : 0.0;
+        if (eff > best_eff + 1e-9 || (eff > best_eff - 1e-9 && waves < best_waves)) {
+            best_eff = eff;
+            best_waves = waves;
+            split = sp;
+        }
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)split, (unsigned)Hkv, (unsigned)B);
     cfg.blockDim = dim3(kAttThreads);
