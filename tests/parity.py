@@ -20,7 +20,7 @@
  * fp16 outputs: max relative error 2e-3 against the oracle's fp64 product,
    relative to max(|y_ref|, 1e-2 * rms(y_ref row)) so that outputs near zero
    (which any rounding order perturbs by more than 2e-3 of themselves) are
-   judged on the row's scale.
+   measured on the row's scale.
 """
 import numpy as np
 
@@ -76,7 +76,7 @@ def check_codes(gpu_packed, gpu_scales, xr, group, max_frac=1e-4):
     t = np.where(s_el > 0, xr / np.where(s_el > 0, s_el, 1.0), 0.0)
     dist = np.abs(t - (np.floor(t) + 0.5))
     assert np.all(dist[flips] < 1e-3), f"code flips away from near-ties (max dist {dist[flips].max():.3e})"
-    # exact ties are judged with the oracle's own scale (fp64 max|x'|/7 per row,
+    # exact ties are decided with the oracle's own scale (fp64 max|x'|/7 per row,
     # or the checked fp16 group scale)
     if group == 0:
         s0 = np.abs(xr).max(axis=1, keepdims=True) / 7.0

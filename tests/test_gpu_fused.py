@@ -54,7 +54,7 @@ def test_fused_equals_separate_and_oracle(q, wid):
     if same_w:
         check_f16_output(yg, yr)
     else:
-        # a few weight codes flipped at near-ties: judge the rows as a whole
+        # a few weight codes flipped at near-ties: assess the rows as a whole
         rel = np.linalg.norm(yg - yr) / np.linalg.norm(yr)
         assert rel <= 2e-3, f"relative Frobenius error {rel:.3e}"
 
