@@ -86,6 +86,24 @@ def test_kv_scores_matches_oracle(q, B, T, H, G):
     _scores_check(q, qh, s, kq, ks)
 
 
+@pytest.mark.parametrize("qscale", [0.0, 1e-6, 1e-3, 300.0])
+def test_kv_scores_query_magnitudes(q, qscale):
+    """Zero, tiny and large queries: the scores must keep their relative
+    accuracy at every scale (a zero query gives exactly zero scores)."""
+    rng = np.random.default_rng(int(qscale * 1e6) % 1000 + 3)
+    B, T, H, G = 1, 200, 2, 8
+    k = rng.standard_normal((B, T, H, 128)).astype(np.float16)
+    s = np.stack([synth.signs(128, 60 + h) for h in range(H)])
+    kq, ks, _, _ = oracle.kv_quant(k, np.zeros_like(k), s)
+    qh = (rng.standard_normal((B, H * G, 128)) * qscale).astype(np.float16)
+    if qscale == 0.0:
+        got = q.quarot_kv_decode_scores(_dev(qh), _dev(s), _dev(kq), _dev(ks.view(np.float16)))
+        _ok(q)
+        np.testing.assert_array_equal(got.cpu().numpy(), 0.0)
+    else:
+        _scores_check(q, qh, s, kq, ks)
+
+
 def test_kv_scores_full_size_sampled(q):
     c = synth.KV_70B
     k, v, qh, s = synth.kv_inputs(c, batch=4)
