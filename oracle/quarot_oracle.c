@@ -29,6 +29,14 @@
  *    (block-diagonal rotations of size 2^n; a normalized Hadamard has a
  *    uniform first row), Knowl 12 (block size 128; a fixed Hadamard with
  *    entries +-1/sqrt(2^n) on the attention path, per-head quantization).
+ *  - The Elamur Research QuaRot summary, References, item 24: Sloane's
+ *    library of Hadamard matrices, for factors whose order is not a power of
+ *    two (here built by Paley's first construction, qo_paley, for the full
+ *    rotation of K = 11008 = 344 * 32, qo_rotate_kron).
+ *  - The rest of a decode attention step (qo_kv_attend): softmax of the
+ *    scores scaled by 1/sqrt(D) over the tokens, then the product with the
+ *    dequantized INT4 value cache (QuaRot abstract: the KV cache in 4 bits;
+ *    DuQuant Knowl 12: softmax outputs are not quantized).
  *
  * Readings where the pages are silent (each is also listed in the design
  * notes): Sylvester order for H_n, normalization 1/sqrt(n), signs applied
