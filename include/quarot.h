@@ -25,9 +25,10 @@
  *
  * Conventions for every entry point:
  *  - All array pointers are DEVICE memory owned by the caller; the library
- *    allocates nothing (except where an entry point says otherwise) and keeps
- *    no state beyond a per-device cache of kernel attributes (and, once the
- *    full Kronecker rotation has run on a device, its 288 KB Hadamard factor).
+ *    allocates nothing and keeps no state beyond a per-device cache of kernel
+ *    attributes and two device arrays compiled into it: the 288 KB Hadamard
+ *    factor of the full Kronecker rotation (filled by that call's first use
+ *    on a device) and the scratch of quarot_rotate_quant_linear_noalloc.
  *  - Every array pointer must be 16-byte aligned; arrays are dense row-major.
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *    default stream).  Argument errors are returned before any launch and
@@ -36,7 +37,8 @@
  *  - fp16 is IEEE binary16.  INT4 codes are two's complement in [-8, 7],
  *    packed two per byte: element 2i in bits 0-3, element 2i+1 in bits 4-7.
  *  - No function throws; none blocks the host except
- *    quarot_get_device_status().
+ *    quarot_get_device_status() (and the first quarot_rotate_quant_kron on a
+ *    device, which copies its factor).
  */
 #ifndef QUAROT_H
 #define QUAROT_H
@@ -105,8 +107,10 @@ quarot_status_t quarot_rotate_quant(const void *x_f16, int64_t M, int64_t K,
  *
  * x_f16 [M, 11008] fp16; signs [11008] int8 (+1 / -1); q_packed [M, 5504]
  * uint8 out; scales fp32 [M] (group 0) or fp16 [M, 86] (group 128) out.
- * K must be 11008 (else QUAROT_ERR_UNSUPPORTED_SHAPE).  The first call on a
- * device allocates and uploads the factor (288 KB, kept until exit).
+ * K must be 11008 (else QUAROT_ERR_UNSUPPORTED_SHAPE).  The factor lives in
+ * a 288 KB device array compiled into the library (nothing is allocated);
+ * the first call on a device fills it with a synchronous host-to-device copy,
+ * so make that first call outside any stream capture.
  */
 quarot_status_t quarot_rotate_quant_kron(const void *x_f16, int64_t M, int64_t K, const int8_t *signs,
                                          int64_t group, uint8_t *q_packed, void *scales, quarot_stream_t stream);
@@ -288,6 +292,43 @@ quarot_status_t quarot_rotate_quant_linear_i8(const void *x_f16, int64_t M, int6
 
 /*
  * ---------------------------------------------------------------------------
+ * The 6-bit variant [QR-S Key points: round-to-nearest is close to lossless
+ * at 6 and 8 bits without calibration; QR-A: higher widths of the same
+ * recipe].  The rotation is the one of quarot_rotate_quant; per row
+ *
+ *   s[m] = max_k |x'[m,k]| / 31 (fp32),  q = rint(x'/s)  (in [-31, 31];
+ *   round half to even; a zero scale gives zero codes)
+ *
+ * Codes are stored one signed byte each, row-major [rows, K], so the INT8
+ * linear layer (quarot_int8_linear, quarot_int8_gemm_s32) takes them as they
+ * are: the tensor cores have no 6-bit integer kind, and a 6-bit code is an
+ * 8-bit code that never leaves [-31, 31] (|acc| <= 961 K, exact).
+ * ---------------------------------------------------------------------------
+ */
+
+/*
+ * quarot_rotate_quant_i6 -- online rotation + 6-bit RTN of activations (or,
+ * offline, of weight rows).  Arguments, limits and layouts as
+ * quarot_rotate_quant_i8: q int8 [M, K] output (codes in [-31, 31]), scales
+ * fp32 [M] output.
+ */
+quarot_status_t quarot_rotate_quant_i6(const void *x_f16, int64_t M, int64_t K, const int8_t *signs,
+                                       int had_block, int8_t *q, float *scales, quarot_stream_t stream);
+
+/*
+ * quarot_rotate_quant_linear_i6 -- the fused online path of one 6-bit linear
+ * layer: quarot_rotate_quant_i6 of x into `workspace`, then
+ * quarot_int8_linear against weights prepared by quarot_rotate_quant_i6.
+ * Arguments as quarot_rotate_quant_linear_i8; the workspace size is
+ * quarot_rotate_quant_linear_i8_workspace(M, K).
+ */
+quarot_status_t quarot_rotate_quant_linear_i6(const void *x_f16, int64_t M, int64_t K, const int8_t *signs,
+                                              int had_block, const int8_t *qw, const float *s_w, int64_t N,
+                                              void *workspace, size_t ws_bytes, void *out_f16,
+                                              quarot_stream_t stream);
+
+/*
+ * ---------------------------------------------------------------------------
  * Asymmetric INT4 with a clipping ratio [DQ-12: per-token asymmetric
  * quantization of activations, per-channel asymmetric quantization of
  * weights, clipping ratios on the extremes (0.9 for activations, 0.8 for
@@ -370,9 +411,9 @@ quarot_status_t quarot_kv_quant(const void *k_f16, const void *v_f16, int64_t B,
  * scores  [B, Hq, T] fp32 output.
  * Limits: D == 128; Hq % Hkv == 0 with Hq / Hkv <= 16; B, T >= 0.
  */
-quarot_status_t quarot_kv_decode_scores(const void *q_f16, int64_t B, int64_t Hq,
-                                        const int8_t *signs, const uint8_t *kq,
-                                        const void *ks_f16, int64_t T, int64_t Hkv, int64_t D,
+quarot_status_t quarot_kv_decode_scores(const void *q_f16, int64_t Hq, const int8_t *signs,
+                                        const uint8_t *kq, const void *ks_f16, int64_t B,
+                                        int64_t T, int64_t Hkv, int64_t D,
                                         float *scores, quarot_stream_t stream);
 
 /*
@@ -394,14 +435,53 @@ quarot_status_t quarot_kv_decode_attend(const float *scores, int64_t B, int64_t 
                                         quarot_stream_t stream);
 
 /*
- * quarot_get_device_status -- synchronizes the current device, then reports
- * (and clears) the library's device-side error word: QUAROT_ERR_DEVICE_TIMEOUT
- * if any kernel since the last call gave up a bounded wait (every wait inside
- * the tensor-core GEMM is bounded in time; on expiry the kernel records the
- * fact, drains its own in-flight work, frees its tensor memory and exits),
- * QUAROT_ERR_CUDA if the synchronization itself failed, else QUAROT_OK.
+ * quarot_get_device_status -- synchronizes `stream` (the whole current device
+ * when stream is NULL), then reports (and clears) the library's device-side
+ * error word: QUAROT_ERR_DEVICE_TIMEOUT if any kernel since the last call
+ * gave up a bounded wait (every wait on a barrier, a copy or the tensor core
+ * is bounded in time; on expiry the kernel records the fact, waits -- again
+ * with a limit -- for the copies and tensor-core work it issued, frees its
+ * tensor memory and exits), QUAROT_ERR_CUDA if the synchronization itself
+ * failed, else QUAROT_OK.  The error word is one per device and process:
+ * with a non-NULL stream, kernels still running on other streams may set it
+ * after the read.
  */
-quarot_status_t quarot_get_device_status(void);
+quarot_status_t quarot_get_device_status(quarot_stream_t stream);
+
+/*
+ * quarot_probe_mma_i8 -- measures the denominator of the linear layers'
+ * roofline (no passage of the pages corresponds to it: the pages time their
+ * kernels on other hardware and give no peak).  On every pair of SMs, one CTA
+ * pair issues `steps` groups of four tcgen05.mma.kind::i8 instructions of the
+ * shape the INT4 and INT8 GEMMs use (M 256, N 256, K 32 each, int32
+ * accumulation in tensor memory), on operands resident in shared memory, and
+ * waits for them; nothing is copied or stored.  *pairs receives the number of
+ * CTA pairs launched, so one call performs pairs * steps * 4 * 2 * 256 * 256
+ * * 32 integer operations; timing the call on `stream` gives the dense INT8
+ * tensor rate.  Limits: 1 <= steps <= 2^22.
+ */
+quarot_status_t quarot_probe_mma_i8(int64_t steps, int64_t *pairs, quarot_stream_t stream);
+
+/*
+ * quarot_test_wait_timeout -- exercises the bounded-wait path of the kernels
+ * (no passage of the pages corresponds to it: it tests the library's failure
+ * reporting, not the method).  It runs the KV-cache value-row quantizer of
+ * quarot_kv_quant (rows of 128 fp16, no rotation, fp16 scale per row) over
+ * `rows` rows, but never issues the copy of tile `withheld_tile` (tiles are
+ * 128 consecutive rows), and bounds every wait by `wait_limit_ns`.  The CTA
+ * that owns the withheld tile gives up its wait after that time, records
+ * QUAROT_ERR_DEVICE_TIMEOUT in the device error word, waits (with the same
+ * bound) for the copies it did issue and exits; nothing is left in flight and
+ * the context stays usable.  The other tiles are quantized as usual; rows of
+ * the aborted CTA from the withheld tile on may be left unwritten.
+ *
+ * v_f16 [rows, 128] fp16; q_packed [rows, 64] uint8 and scales_f16 [rows]
+ * fp16 outputs.  Limits: 1 <= rows < 2^31 - 128; 0 <= withheld_tile <
+ * ceil(rows / 128); 1e5 <= wait_limit_ns <= 2e9.  Returns the launch status;
+ * quarot_get_device_status() then reports the timeout.
+ */
+quarot_status_t quarot_test_wait_timeout(const void *v_f16, int64_t rows, uint8_t *q_packed, void *scales_f16,
+                                         int64_t withheld_tile, uint64_t wait_limit_ns, quarot_stream_t stream);
 
 /* Static, human-readable name of a status code. */
 const char *quarot_status_string(quarot_status_t status);

@@ -40,15 +40,19 @@ _SIGS = {
     "quarot_int8_gemm_s32": ([_P, _I64, _P, _I64, _I64, _P, _P], _INT),
     "quarot_rotate_quant_linear_i8_workspace": ([_I64, _I64], _SZ),
     "quarot_rotate_quant_linear_i8": ([_P, _I64, _I64, _P, _INT, _P, _P, _I64, _P, _SZ, _P, _P], _INT),
+    "quarot_rotate_quant_i6": ([_P, _I64, _I64, _P, _INT, _P, _P, _P], _INT),
+    "quarot_rotate_quant_linear_i6": ([_P, _I64, _I64, _P, _INT, _P, _P, _I64, _P, _SZ, _P, _P], _INT),
     "quarot_rotate_quant_asym": ([_P, _I64, _I64, _P, _INT, ctypes.c_float, _P, _P, _P, _P, _P], _INT),
     "quarot_uint4_gemm_s32": ([_P, _I64, _P, _I64, _I64, _P, _P], _INT),
     "quarot_int4_linear_asym": ([_P, _P, _P, _P, _I64, _P, _P, _P, _P, _I64, _I64, _P, _P], _INT),
     "quarot_kv_quant": ([_P, _P, _I64, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P], _INT),
-    "quarot_kv_decode_scores": ([_P, _I64, _I64, _P, _P, _P, _I64, _I64, _I64, _P, _P], _INT),
+    "quarot_kv_decode_scores": ([_P, _I64, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P], _INT),
     "quarot_rotate_quant_kron": ([_P, _I64, _I64, _P, _I64, _P, _P, _P], _INT),
     "quarot_kron_factor": ([_I64, _P], _INT),
     "quarot_kv_decode_attend": ([_P, _I64, _I64, _P, _P, _I64, _I64, _I64, _P, _P], _INT),
-    "quarot_get_device_status": ([], _INT),
+    "quarot_probe_mma_i8": ([_I64, _P, _P], _INT),
+    "quarot_test_wait_timeout": ([_P, _I64, _P, _P, _I64, ctypes.c_uint64, _P], _INT),
+    "quarot_get_device_status": ([_P], _INT),
     "quarot_status_string": ([_INT], ctypes.c_char_p),
     "quarot_last_error": ([], ctypes.c_char_p),
 }
@@ -240,6 +244,38 @@ def quarot_rotate_quant_linear_i8(x: torch.Tensor, signs: torch.Tensor, qw: torc
     return out
 
 
+def quarot_rotate_quant_i6(x: torch.Tensor, signs: torch.Tensor, had_block: int = 0,
+                           q: Optional[torch.Tensor] = None, scales: Optional[torch.Tensor] = None, stream=None):
+    """x fp16 [M, K] -> (q int8 [M, K] in [-31, 31], scales fp32 [M]): the 6-bit variant."""
+    M, K = x.shape
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if scales is None:
+        scales = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _check("quarot_rotate_quant_i6",
+           lib.quarot_rotate_quant_i6(_ptr(x), M, K, _ptr(signs), had_block, _ptr(q), _ptr(scales),
+                                      _stream(stream)))
+    return q, scales
+
+
+def quarot_rotate_quant_linear_i6(x: torch.Tensor, signs: torch.Tensor, qw: torch.Tensor, s_w: torch.Tensor,
+                                  had_block: int = 0, workspace: Optional[torch.Tensor] = None,
+                                  out: Optional[torch.Tensor] = None, stream=None):
+    """Fused online 6-bit path: rotate + 6-bit quantize x, then the INT8 linear; fp16 [M, N]."""
+    M, K = x.shape
+    N = qw.shape[0]
+    need = quarot_rotate_quant_linear_i8_workspace(M, K)
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=x.device)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=x.device)
+    _check("quarot_rotate_quant_linear_i6",
+           lib.quarot_rotate_quant_linear_i6(_ptr(x), M, K, _ptr(signs), had_block, _ptr(qw), _ptr(s_w), N,
+                                             _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                             _ptr(out), _stream(stream)))
+    return out
+
+
 def quarot_rotate_quant_asym(x: torch.Tensor, signs: torch.Tensor, clip: float, had_block: int = 0, q=None, d=None,
                              z=None, r=None, stream=None):
     """x fp16 [M, K] -> (q_packed uint8 [M, K/2] unsigned nibbles, steps fp32 [M],
@@ -303,7 +339,7 @@ def quarot_kv_decode_scores(q: torch.Tensor, signs: torch.Tensor, kq: torch.Tens
     if scores is None:
         scores = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
     _check("quarot_kv_decode_scores",
-           lib.quarot_kv_decode_scores(_ptr(q), B, Hq, _ptr(signs), _ptr(kq), _ptr(ks), T, H, D, _ptr(scores),
+           lib.quarot_kv_decode_scores(_ptr(q), Hq, _ptr(signs), _ptr(kq), _ptr(ks), B, T, H, D, _ptr(scores),
                                        _stream(stream)))
     return scores
 
@@ -342,5 +378,31 @@ def quarot_kv_decode_attend(scores: torch.Tensor, vq: torch.Tensor, vs: torch.Te
     return out
 
 
-def quarot_get_device_status() -> int:
-    return int(lib.quarot_get_device_status())
+def quarot_probe_mma_i8(steps: int, stream=None) -> int:
+    """Launches the dense INT8 tensor-pipe probe; returns the integer
+    operations it performs (time it on the stream with CUDA events)."""
+    pairs = ctypes.c_int64(0)
+    _check("quarot_probe_mma_i8", lib.quarot_probe_mma_i8(steps, ctypes.byref(pairs), _stream(stream)))
+    return int(pairs.value) * steps * 4 * 2 * 256 * 256 * 32
+
+
+def quarot_test_wait_timeout(v: torch.Tensor, withheld_tile: int, wait_limit_ns: int,
+                             q: Optional[torch.Tensor] = None, scales: Optional[torch.Tensor] = None, stream=None):
+    """The value-row quantizer over v fp16 [rows, 128] with the copy of one
+    128-row tile withheld and every wait bounded by wait_limit_ns (tests the
+    timeout path); returns (q [rows, 64], scales fp16 [rows])."""
+    rows = v.shape[0]
+    if q is None:
+        q = torch.zeros((rows, 64), dtype=torch.uint8, device=v.device)
+    if scales is None:
+        scales = torch.zeros((rows,), dtype=torch.float16, device=v.device)
+    _check("quarot_test_wait_timeout",
+           lib.quarot_test_wait_timeout(_ptr(v), rows, _ptr(q), _ptr(scales), withheld_tile, wait_limit_ns,
+                                        _stream(stream)))
+    return q, scales
+
+
+def quarot_get_device_status(stream=None) -> int:
+    """Synchronizes `stream` (the whole device when None) and returns, then
+    clears, the library's device error word (0 = no bounded wait gave up)."""
+    return int(lib.quarot_get_device_status(None if stream is None else _stream(stream)))

@@ -22,6 +22,31 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
     return t;
 }
 
+// Waits until the phase of the mbarrier at shared address `bar` with parity
+// `parity` has completed, for at most `limit_ns`; on expiry records a timeout
+// in the device status word and returns false.  Used to drain copies a
+// thread issued before it exits (the wait ignores any abort of the caller).
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns)
+{
+    uint32_t done;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (done)
+            return true;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            record_timeout();
+            return false;
+        }
+    }
+}
+
 // Round-to-nearest-even of v into the low mantissa bits of a float: for
 // |v| < 2^22, 1.5*2^23 + v has unit spacing, so the single rounding of the
 // addition is the integer rounding (ties to even) and the low 4 bits of the

@@ -80,6 +80,7 @@ int8_gemm_pair_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_
     const uint32_t bar_drain = bar_acce + 16;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + S::kMiscOffset);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + S::kMiscOffset + 4);
+    int *peer_steps = reinterpret_cast<int *>(smem + S::kMiscOffset + 8);   // leader: steps the peer issued
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -103,6 +104,7 @@ int8_gemm_pair_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_
         }
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
+        *peer_steps = -1;
         mbar_fence_init();
     }
     if (warp == S::kMmaWarp) {
@@ -144,16 +146,38 @@ int8_gemm_pair_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_
                         gemm_tile_coords(cluster + lt * nclusters, a.tiles_m, a.tiles_n, mb, nb);
                 }
             }
-            // In a normal run every copy lands before the pair exits: its bytes
-            // count on a leader barrier that the MMA thread waits on before the
-            // final cluster barrier.  After an abort, copies
-            // issued into stages the MMA never consumed may still be in flight,
-            // and the peer cannot wait on the leader's barriers; both CTAs then
-            // give them a fixed grace time (far longer than a copy) before the
-            // final cluster barrier lets the pair exit.
-            if (step < total) {
+            // Every copy either CTA issued lands before the pair passes the
+            // final cluster barrier.  All of them count on the leader's stage
+            // barriers, so the peer reports how many steps it issued and the
+            // leader waits for the last kStages steps of either CTA (earlier
+            // ones were consumed before their stages were refilled).  In a
+            // normal run both issued every step and those phases are complete.
+            // After an abort the two counts may differ: a step only the peer
+            // issued gets the leader's missing arrival (declaring the peer's
+            // bytes), a step only the leader issued gets the peer's declared
+            // bytes completed without a copy, so each phase completes once the
+            // copies actually issued have landed.
+            if (!leader) {
+                st_release_cluster_u32(mapa_shared(smem_u32(peer_steps), 0), (uint32_t)step);
+            } else {
+                int peer = -1;
                 const uint64_t t0 = globaltimer_ns();
-                while (globaltimer_ns() - t0 < 1000000ull) {
+                while ((peer = (int)ld_acquire_cluster_u32(smem_u32(peer_steps))) < 0) {
+                    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                        record_timeout();
+                        break;
+                    }
+                }
+                if (peer >= 0) {
+                    const int hi = max(step, peer);
+                    for (int j = max(0, hi - S::kStages); j < hi; ++j) {
+                        const uint32_t fb = bar_full + 8 * (j % S::kStages);
+                        if (j >= step)
+                            mbar_arrive_expect_tx(fb, S::kStageBytes);
+                        else if (j >= peer)
+                            mbar_complete_tx(fb, S::kStageBytes);
+                        gemm_wait_drain(fb, (uint32_t)(j / S::kStages) & 1);
+                    }
                 }
             }
         }

@@ -255,11 +255,12 @@ kron_quant_kernel(const __grid_constant__ CUtensorMap tma_h,     // H^T, fp16 [3
                                   x + (row0 + r) * kKronK + (int64_t)kb * 64 * kKronN, bytes, bar_xfull + 8 * s);
                 }
             }
-            if (!ok) {
-                const uint64_t t0 = globaltimer_ns();
-                while (globaltimer_ns() - t0 < 1000000ull) {
-                }
-            }
+            // every copy issued lands before the CTA can exit: at most the
+            // last kKronXStages steps can still be in flight (each stage was
+            // consumed before it was refilled)
+            for (int j = step - kKronXStages; j < step; ++j)
+                if (j >= 0)
+                    gemm_wait_drain(bar_xfull + 8 * (j % kKronXStages), (uint32_t)(j / kKronXStages) & 1);
         }
         __syncwarp();
     } else if (warp == kKronAWarp) {
@@ -279,11 +280,10 @@ kron_quant_kernel(const __grid_constant__ CUtensorMap tma_h,     // H^T, fp16 [3
                         mbar_arrive_expect_tx(bar_afull + 8 * s, kKronBlock);
                         tma_load_2d(sbase + S::kAOff + s * kKronBlock, &tma_h, kb * 64, t * 128, bar_afull + 8 * s);
                     }
-            if (!ok) {
-                const uint64_t t0 = globaltimer_ns();
-                while (globaltimer_ns() - t0 < 1000000ull) {
-                }
-            }
+            // as for x: the copies of the last kKronAStages steps land before exit
+            for (int j = step - kKronAStages; j < step; ++j)
+                if (j >= 0)
+                    gemm_wait_drain(bar_afull + 8 * (j % kKronAStages), (uint32_t)(j / kKronAStages) & 1);
         }
         __syncwarp();
     } else if (warp == kKronMmaWarp) {

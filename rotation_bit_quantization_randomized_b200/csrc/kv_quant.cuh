@@ -37,7 +37,9 @@ kv_quant_tma_kernel(const __grid_constant__ CUtensorMap tmap,   // fp16 [rows, 1
                     int64_t rows, int hkv, const int8_t *__restrict__ signs,
                     uint8_t *__restrict__ q,                    // [rows, 64]
                     __half *__restrict__ scales,                // [rows]
-                    float scale_mul, float sqrt_n)
+                    float scale_mul, float sqrt_n,
+                    uint64_t wait_limit_ns,                     // bound of every wait
+                    int64_t withheld_tile)                      // tile whose copy is never issued (-1: none)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -56,7 +58,11 @@ kv_quant_tma_kernel(const __grid_constant__ CUtensorMap tmap,   // fp16 [rows, 1
     }
     __syncthreads();
 
+    int issued = 0;                       // thread 0: tiles whose copies were issued (in tile order)
     auto issue = [&](int64_t tile, int s) {
+        ++issued;
+        if (tile == withheld_tile)
+            return;                       // only the timeout test withholds a copy
         const uint32_t dst = sbase + s * kKvStageBytes;
         mbar_arrive_expect_tx(bar_full + 8 * s, kKvStageBytes);
         tma_load_2d(dst, &tmap, 0, (int)(tile * kKvTileRows), bar_full + 8 * s);
@@ -87,7 +93,7 @@ kv_quant_tma_kernel(const __grid_constant__ CUtensorMap tmap,   // fp16 [rows, 1
         if (!mbar_try_wait(bar_full + 8 * s, parity)) {
             const uint64_t t0 = globaltimer_ns();
             while (!mbar_try_wait(bar_full + 8 * s, parity)) {
-                if (globaltimer_ns() - t0 > kKvWaitLimitNs) {
+                if (globaltimer_ns() - t0 > wait_limit_ns) {
                     record_timeout();
                     ok = false;
                     break;
@@ -131,12 +137,11 @@ kv_quant_tma_kernel(const __grid_constant__ CUtensorMap tmap,   // fp16 [rows, 1
             scales[row] = s16;
         quant_pack_store<128>(v, r, q + (valid ? row : 0) * 64, valid);
     }
-    // copies issued beyond the consumed tiles (abort only) must land before exit
-    if (t == 0 && !ok) {
-        const uint64_t t0 = globaltimer_ns();
-        while (globaltimer_ns() - t0 < 1000000ull) {
-        }
-    }
+    // copies issued beyond the consumed tiles (abort only) land before exit:
+    // iterations it .. issued - 1 had their copies issued but were not waited for
+    if (t == 0)
+        for (int j = it; j < issued; ++j)
+            mbar_wait_drain(bar_full + 8 * (j % kKvStages), (uint32_t)(j / kKvStages) & 1, wait_limit_ns);
 }
 
 }  // namespace quarot

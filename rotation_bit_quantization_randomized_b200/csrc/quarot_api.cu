@@ -11,6 +11,7 @@
 #include "kv_attend.cuh"
 #include "kv_quant.cuh"
 #include "kv_scores.cuh"
+#include "mma_peak.cuh"
 #include "rotate_quant.cuh"
 
 #include <cuda.h>
@@ -150,7 +151,7 @@ quarot_status_t check_rotate_args(const void *x, int64_t M, int64_t K, const int
 }
 
 // qmax of a code width: the largest code magnitude of the symmetric RTN.
-constexpr double qmax_of(int bits) { return bits == 8 ? 127.0 : 7.0; }
+constexpr double qmax_of(int bits) { return (double)code_qmax(bits); }
 
 template <int LOGN, int GROUP, int BITS, bool ASYM = false>
 quarot_status_t launch_fwht(const void *x, int64_t M, const int8_t *signs, uint8_t *q, void *scales,
@@ -223,7 +224,7 @@ quarot_status_t launch_block(const void *x, int64_t M, int64_t K, const int8_t *
     return after_launch("block128_quant_kernel launch");
 }
 
-// bits == 8 implies group == 0 (checked by the callers).
+// bits 6 and 8 imply group == 0 (checked by the callers).
 quarot_status_t rotate_quant_launch(const void *x, int64_t M, int64_t K, const int8_t *signs, int had_block,
                                     int group, uint8_t *q, void *scales, cudaStream_t st, int bits = 4)
 {
@@ -237,6 +238,8 @@ quarot_status_t rotate_quant_launch(const void *x, int64_t M, int64_t K, const i
         const int logn = ilog2(K);
         if (bits == 8)
             return dispatch_fwht<0, 8>(logn, x, M, signs, q, scales, st, dev, sms);
+        if (bits == 6)
+            return dispatch_fwht<0, 6>(logn, x, M, signs, q, scales, st, dev, sms);
         return group == 0 ? dispatch_fwht<0, 4>(logn, x, M, signs, q, scales, st, dev, sms)
                           : dispatch_fwht<128, 4>(logn, x, M, signs, q, scales, st, dev, sms);
     }
@@ -244,6 +247,8 @@ quarot_status_t rotate_quant_launch(const void *x, int64_t M, int64_t K, const i
     const float sq = (float)std::sqrt(128.0);
     if (bits == 8)
         return launch_block<true, 0, 8>(x, M, K, signs, q, scales, mul, sq, st, dev, sms);
+    if (bits == 6)
+        return launch_block<true, 0, 6>(x, M, K, signs, q, scales, mul, sq, st, dev, sms);
     return group == 0 ? launch_block<true, 0>(x, M, K, signs, q, scales, mul, sq, st, dev, sms)
                       : launch_block<true, 128>(x, M, K, signs, q, scales, mul, sq, st, dev, sms);
 }
@@ -599,7 +604,11 @@ void paley344(int8_t *H)
     }
 }
 
-// H^T as fp16, zero-padded to 384 x 384 (the MMA operand), once per device.
+// H^T as fp16, zero-padded to 384 x 384 (the MMA operand): an array compiled
+// into the library (nothing is allocated), filled once per device by a
+// synchronous copy with that device current; the kernels get the address
+// cudaGetSymbolAddress returns for that device.
+static __device__ __align__(256) uint16_t g_kron_ht[kKronAPad * kKronAPad];
 std::mutex g_kron_mutex;
 void *g_kron_factor[kMaxDevices] = {};
 
@@ -613,15 +622,13 @@ quarot_status_t kron_factor_device(int dev, const void *&ptr)
         for (int ap = 0; ap < kKronM; ++ap)
             for (int a = 0; a < kKronM; ++a)
                 Ht[(size_t)ap * kKronAPad + a] = H[(size_t)a * kKronM + ap] > 0 ? 0x3C00 : 0xBC00;
-        void *d = nullptr;
-        cudaError_t e = cudaMalloc(&d, Ht.size() * 2);
+        cudaError_t e = cudaMemcpyToSymbol(g_kron_ht, Ht.data(), Ht.size() * 2);
         if (e != cudaSuccess)
-            return cuda_fail(e, "cudaMalloc (Hadamard factor)");
-        e = cudaMemcpy(d, Ht.data(), Ht.size() * 2, cudaMemcpyHostToDevice);
-        if (e != cudaSuccess) {
-            cudaFree(d);
-            return cuda_fail(e, "cudaMemcpy (Hadamard factor)");
-        }
+            return cuda_fail(e, "cudaMemcpyToSymbol (Hadamard factor)");
+        void *d = nullptr;
+        e = cudaGetSymbolAddress(&d, g_kron_ht);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cudaGetSymbolAddress (Hadamard factor)");
         g_kron_factor[dev] = d;
     }
     ptr = g_kron_factor[dev];
@@ -743,7 +750,8 @@ quarot_status_t kv_map(CUtensorMap &map, const void *base, int64_t rows)
 // The staged KV-write kernel over `rows` rows of 128 elements (Hkv divides 128).
 template <bool ROTATE>
 quarot_status_t launch_kv_tma(const void *x, int64_t rows, int hkv, const int8_t *signs, uint8_t *q, void *scales,
-                              float scale_mul, float sqrt_n, cudaStream_t st, int dev, int sms)
+                              float scale_mul, float sqrt_n, cudaStream_t st, int dev, int sms,
+                              uint64_t wait_limit_ns = kKvWaitLimitNs, int64_t withheld_tile = -1)
 {
     auto kern = kv_quant_tma_kernel<ROTATE>;
     int per_sm = 0;
@@ -757,7 +765,7 @@ quarot_status_t launch_kv_tma(const void *x, int64_t rows, int hkv, const int8_t
     const int64_t tiles = (rows + kKvTileRows - 1) / kKvTileRows;
     const int grid = (int)std::min<int64_t>(tiles, (int64_t)sms * per_sm);
     kern<<<grid, kKvTileRows, kKvSmemBytes, st>>>(map, rows, hkv, signs, q, static_cast<__half *>(scales), scale_mul,
-                                                 sqrt_n);
+                                                 sqrt_n, wait_limit_ns, withheld_tile);
     return after_launch("kv_quant_tma_kernel launch");
 }
 
@@ -907,6 +915,16 @@ quarot_status_t quarot_rotate_quant_i8(const void *x_f16, int64_t M, int64_t K, 
                                (cudaStream_t)stream, 8);
 }
 
+quarot_status_t quarot_rotate_quant_i6(const void *x_f16, int64_t M, int64_t K, const int8_t *signs, int had_block,
+                                       int8_t *q, float *scales, quarot_stream_t stream)
+{
+    quarot_status_t s = check_rotate_args(x_f16, M, K, signs, had_block, 0, q, scales);
+    if (s != QUAROT_OK || M == 0)
+        return s;
+    return rotate_quant_launch(x_f16, M, K, signs, had_block, 0, reinterpret_cast<uint8_t *>(q), scales,
+                               (cudaStream_t)stream, 6);
+}
+
 quarot_status_t quarot_int8_linear(const int8_t *qa, const float *s_a, int64_t M, const int8_t *qw, const float *s_w,
                                    int64_t N, int64_t K, void *out_f16, quarot_stream_t stream)
 {
@@ -939,10 +957,13 @@ size_t quarot_rotate_quant_linear_i8_workspace(int64_t M, int64_t K)
     return align256((size_t)M * (size_t)K) + align256((size_t)M * 4);
 }
 
-quarot_status_t quarot_rotate_quant_linear_i8(const void *x_f16, int64_t M, int64_t K, const int8_t *signs,
-                                              int had_block, const int8_t *qw, const float *s_w, int64_t N,
-                                              void *workspace, size_t ws_bytes, void *out_f16,
-                                              quarot_stream_t stream)
+namespace {
+// The fused path of the byte-code variants (bits 6 or 8): quantizer into the
+// workspace, then the INT8 tensor-core GEMM as its programmatic dependent.
+quarot_status_t rotate_quant_linear_bytes(const void *x_f16, int64_t M, int64_t K, const int8_t *signs,
+                                          int had_block, const int8_t *qw, const float *s_w, int64_t N,
+                                          void *workspace, size_t ws_bytes, void *out_f16, quarot_stream_t stream,
+                                          int bits)
 {
     quarot_status_t s = check_rotate_args(x_f16, M, K, signs, had_block, 0, workspace, workspace);
     if (s != QUAROT_OK)
@@ -958,10 +979,29 @@ quarot_status_t quarot_rotate_quant_linear_i8(const void *x_f16, int64_t M, int6
     int8_t *qa = static_cast<int8_t *>(workspace);
     float *sa = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + align256((size_t)M * (size_t)K));
     cudaStream_t st = (cudaStream_t)stream;
-    s = rotate_quant_launch(x_f16, M, K, signs, had_block, 0, reinterpret_cast<uint8_t *>(qa), sa, st, 8);
+    s = rotate_quant_launch(x_f16, M, K, signs, had_block, 0, reinterpret_cast<uint8_t *>(qa), sa, st, bits);
     if (s != QUAROT_OK)
         return s;
     return linear8_launch(qa, sa, M, qw, s_w, N, K, out_f16, st, true);
+}
+}  // namespace
+
+quarot_status_t quarot_rotate_quant_linear_i8(const void *x_f16, int64_t M, int64_t K, const int8_t *signs,
+                                              int had_block, const int8_t *qw, const float *s_w, int64_t N,
+                                              void *workspace, size_t ws_bytes, void *out_f16,
+                                              quarot_stream_t stream)
+{
+    return rotate_quant_linear_bytes(x_f16, M, K, signs, had_block, qw, s_w, N, workspace, ws_bytes, out_f16, stream,
+                                     8);
+}
+
+quarot_status_t quarot_rotate_quant_linear_i6(const void *x_f16, int64_t M, int64_t K, const int8_t *signs,
+                                              int had_block, const int8_t *qw, const float *s_w, int64_t N,
+                                              void *workspace, size_t ws_bytes, void *out_f16,
+                                              quarot_stream_t stream)
+{
+    return rotate_quant_linear_bytes(x_f16, M, K, signs, had_block, qw, s_w, N, workspace, ws_bytes, out_f16, stream,
+                                     6);
 }
 
 quarot_status_t quarot_rotate_quant_asym(const void *x_f16, int64_t M, int64_t K, const int8_t *signs, int had_block,
@@ -1077,8 +1117,8 @@ quarot_status_t quarot_kv_quant(const void *k_f16, const void *v_f16, int64_t B,
                                     info->sm_count);
 }
 
-quarot_status_t quarot_kv_decode_scores(const void *q_f16, int64_t B, int64_t Hq, const int8_t *signs,
-                                        const uint8_t *kq, const void *ks_f16, int64_t T, int64_t Hkv, int64_t D,
+quarot_status_t quarot_kv_decode_scores(const void *q_f16, int64_t Hq, const int8_t *signs, const uint8_t *kq,
+                                        const void *ks_f16, int64_t B, int64_t T, int64_t Hkv, int64_t D,
                                         float *scores, quarot_stream_t stream)
 {
     if (B < 0 || T < 0 || Hkv <= 0 || Hq <= 0)
@@ -1196,11 +1236,70 @@ quarot_status_t quarot_kv_decode_attend(const float *scores, int64_t B, int64_t 
     return after_launch("kv_attend_kernel launch");
 }
 
-quarot_status_t quarot_get_device_status(void)
+quarot_status_t quarot_probe_mma_i8(int64_t steps, int64_t *pairs, quarot_stream_t stream)
 {
-    cudaError_t e = cudaDeviceSynchronize();
+    if (steps < 1 || steps > (int64_t(1) << 22))
+        return fail(QUAROT_ERR_INVALID_ARG, "steps must lie in [1, 2^22]");
+    if (!pairs)
+        return fail(QUAROT_ERR_INVALID_ARG, "null pointer");
+    int dev;
+    DeviceInfo *info;
+    quarot_status_t s = current_device(dev, info);
+    if (s != QUAROT_OK)
+        return s;
+    using S = MmaPeakShape;
+    int per_sm = 0;
+    s = kernel_occupancy(mma_peak_i8_kernel, dev, S::kThreads, S::kSmemBytes, per_sm);
+    if (s != QUAROT_OK)
+        return s;
+    const int clusters = info->sm_count / 2;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * clusters);
+    cfg.blockDim = dim3(S::kThreads);
+    cfg.dynamicSmemBytes = S::kSmemBytes;
+    cfg.stream = (cudaStream_t)stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, mma_peak_i8_kernel, steps);
     if (e != cudaSuccess)
-        return cuda_fail(e, "cudaDeviceSynchronize");
+        return cuda_fail(e, "mma_peak_i8_kernel launch");
+    *pairs = clusters;
+    return after_launch("mma_peak_i8_kernel launch");
+}
+
+quarot_status_t quarot_test_wait_timeout(const void *v_f16, int64_t rows, uint8_t *q_packed, void *scales_f16,
+                                         int64_t withheld_tile, uint64_t wait_limit_ns, quarot_stream_t stream)
+{
+    if (rows <= 0 || rows >= (int64_t(1) << 31) - kKvTileRows)
+        return fail(QUAROT_ERR_INVALID_ARG, "rows must lie in [1, 2^31 - 128)");
+    const int64_t tiles = (rows + kKvTileRows - 1) / kKvTileRows;
+    if (withheld_tile < 0 || withheld_tile >= tiles)
+        return fail(QUAROT_ERR_INVALID_ARG, "withheld_tile must name one of the tiles of 128 rows");
+    if (wait_limit_ns < 100000ull || wait_limit_ns > kKvWaitLimitNs)
+        return fail(QUAROT_ERR_INVALID_ARG, "wait_limit_ns must lie in [1e5, 2e9]");
+    if (!v_f16 || !q_packed || !scales_f16)
+        return fail(QUAROT_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(v_f16) || !aligned16(q_packed) || !aligned16(scales_f16))
+        return fail(QUAROT_ERR_MISALIGNED, "rows, codes and scales must be 16-byte aligned");
+    int dev;
+    DeviceInfo *info;
+    quarot_status_t s = current_device(dev, info);
+    if (s != QUAROT_OK)
+        return s;
+    return launch_kv_tma<false>(v_f16, rows, 1, nullptr, q_packed, scales_f16, (float)(1.0 / 7.0), 1.0f,
+                                (cudaStream_t)stream, dev, info->sm_count, wait_limit_ns, withheld_tile);
+}
+
+quarot_status_t quarot_get_device_status(quarot_stream_t stream)
+{
+    cudaError_t e = stream ? cudaStreamSynchronize((cudaStream_t)stream) : cudaDeviceSynchronize();
+    if (e != cudaSuccess)
+        return cuda_fail(e, stream ? "cudaStreamSynchronize" : "cudaDeviceSynchronize");
     int v = 0;
     e = cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int));
     if (e != cudaSuccess)

@@ -39,6 +39,11 @@
 
 namespace quarot {
 
+// Largest code magnitude of the symmetric RTN at a code width: 2^(b-1) - 1.
+// 4-bit codes are packed two per byte; 6- and 8-bit codes are stored one
+// signed byte each.
+__host__ __device__ constexpr float code_qmax(int bits) { return bits == 8 ? 127.0f : bits == 6 ? 31.0f : 7.0f; }
+
 constexpr int kFwhtThreads = 64;
 constexpr int kBlockThreads = 128;
 
@@ -123,10 +128,11 @@ struct AsymOut {
     float clip;          // clipping ratio of the row's min and max
 };
 
-// Rounds 128 values of one thread to signed 8-bit codes and stores the 128
-// bytes (the 8-bit variant of the same RTN).  r = 127 / max|y| of the row, so
-// |v r| <= 127 (1 + 2^-23) and no clamp is needed; the low byte of the bit
-// pattern of fma(v, r, 1.5 * 2^23) is the two's-complement code.
+// Rounds 128 values of one thread to signed codes of one byte each and stores
+// the 128 bytes (the 6- and 8-bit variants of the same RTN).  r = qmax / max|y|
+// of the row (qmax = 31 or 127), so |v r| <= qmax (1 + 2^-23) and no clamp is
+// needed; the low byte of the bit pattern of fma(v, r, 1.5 * 2^23) is the
+// two's-complement code.
 __device__ __forceinline__ void quant_store_i8(const float (&v)[128], float r, int8_t *dst, bool valid)
 {
 #pragma unroll
@@ -193,10 +199,10 @@ fwht_quant_kernel(const uint32_t *__restrict__ x,      // [M, K/2] fp16 pairs
                   AsymOut asym)                        // asymmetric variant only
 {
     static_assert(LOGN >= 8 && LOGN <= 13, "full transform covers 256..8192");
-    static_assert(BITS == 4 || (BITS == 8 && GROUP == 0), "8-bit codes use one scale per row");
+    static_assert(BITS == 4 || ((BITS == 6 || BITS == 8) && GROUP == 0), "6- and 8-bit codes use one scale per row");
     static_assert(!ASYM || (GROUP == 0 && BITS == 4), "asymmetric codes: 4 bits, one step per row");
     using S = FwhtSmem<LOGN>;
-    constexpr float kQmax = BITS == 8 ? 127.0f : 7.0f;
+    constexpr float kQmax = code_qmax(BITS);
     constexpr int N = S::N;
     constexpr int T = S::T;
     constexpr int R = S::R;
@@ -238,7 +244,7 @@ fwht_quant_kernel(const uint32_t *__restrict__ x,      // [M, K/2] fp16 pairs
 
     const uint32_t *stage = reinterpret_cast<const uint32_t *>(fwht_smem + rl * S::kStageRowBytes);
     int it = 0;
-    bool ok = true;
+    bool ok = true, aborted = false;
     for (int64_t row0 = (int64_t)blockIdx.x * R; row0 < M; row0 += stride, ++it) {
         const int64_t row = row0 + rl;
         const bool valid = row < M;
@@ -253,8 +259,10 @@ fwht_quant_kernel(const uint32_t *__restrict__ x,      // [M, K/2] fp16 pairs
                 }
             }
         }
-        if (!__syncthreads_and(ok))
+        if (!__syncthreads_and(ok)) {
+            aborted = true;
             break;
+        }
 
         // ---- phase A: register r = 2 j + b holds element (j << SH) + 2 tr + b
         // (rows past M were not copied: their slots hold stale data, and
@@ -368,17 +376,16 @@ fwht_quant_kernel(const uint32_t *__restrict__ x,      // [M, K/2] fp16 pairs
             if (valid)
                 reinterpret_cast<__half *>(scales)[row * (N / 128) + tr] = s16;
         }
-        if (BITS == 8)
+        if (BITS != 4)
             quant_store_i8(v, r, reinterpret_cast<int8_t *>(q) + (valid ? row : 0) * N + tr * 128, valid);
         else
             quant_pack_store<GROUP>(v, r, q + (valid ? row : 0) * (N / 2) + tr * 64, valid);
     }
-    // after an abort, a copy may still be in flight into this CTA's memory
-    if (!ok && tid == 0) {
-        const uint64_t t0 = globaltimer_ns();
-        while (globaltimer_ns() - t0 < 1000000ull) {
-        }
-    }
+    // after an abort the copy of the iteration that was given up was issued
+    // (in the previous iteration, or before the loop) and may still be in
+    // flight into this CTA's memory: wait for it before exiting
+    if (aborted && tid == 0)
+        mbar_wait_drain(bar, (uint32_t)it & 1, 2000000000ull);
     // a dependent GEMM launched with programmatic serialization may start now
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
@@ -422,9 +429,9 @@ block128_quant_kernel(const uint4 *__restrict__ x,     // [M, K] fp16, 8 per uin
                       void *__restrict__ scales,
                       float scale_mul, float sqrt_n)
 {
-    static_assert(BITS == 4 || (BITS == 8 && GROUP == 0), "8-bit codes use one scale per row");
-    constexpr float kQmax = BITS == 8 ? 127.0f : 7.0f;
-    constexpr int kCodeBytes = BITS == 8 ? 128 : 64;   // bytes of one 128-block's codes
+    static_assert(BITS == 4 || ((BITS == 6 || BITS == 8) && GROUP == 0), "6- and 8-bit codes use one scale per row");
+    constexpr float kQmax = code_qmax(BITS);
+    constexpr int kCodeBytes = BITS == 4 ? 64 : 128;   // bytes of one 128-block's codes
     constexpr int BPT = MULTI ? 4 : 1;                 // blocks per thread, at most
     __shared__ unsigned int rowmax[kBlockThreads];
     __shared__ uint32_t sgn_multi[MULTI ? BPT * 4 * kBlockThreads : 1];   // [block i][word][thread]
@@ -463,7 +470,7 @@ block128_quant_kernel(const uint4 *__restrict__ x,     // [M, K] fp16, 8 per uin
         const int64_t row = row0 + rl;
         const bool row_ok = active && row < M;
         const uint4 *xrow = x + (row_ok ? row : 0) * (K / 8);
-        uint8_t *qrow = q + (row_ok ? row : 0) * ((int64_t)K * BITS / 8);
+        uint8_t *qrow = q + (row_ok ? row : 0) * ((int64_t)K * kCodeBytes / 128);
 
         if (GROUP != 0) {
             // independent blocks
@@ -514,7 +521,7 @@ block128_quant_kernel(const uint4 *__restrict__ x,     // [M, K] fp16, 8 per uin
             if (row_ok && b0 == 0)
                 reinterpret_cast<float *>(scales)[row] = amax * scale_mul;
             auto store = [&](uint8_t *dst, bool ok) {
-                if (BITS == 8)
+                if (BITS != 4)
                     quant_store_i8(v, r, reinterpret_cast<int8_t *>(dst), ok);
                 else
                     quant_pack_store<0>(v, r, dst, ok);

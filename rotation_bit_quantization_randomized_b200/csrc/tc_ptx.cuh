@@ -41,6 +41,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
+// Completes `bytes` of the transaction count of `bar`'s current phase without
+// a copy (accounts for bytes that were declared but will never be copied).
+__device__ __forceinline__ void mbar_complete_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
 // Arrives on `bar` and adds `bytes` to the transaction count the phase waits for.
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes)
 {
@@ -219,6 +226,21 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank)
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr)
 {
     asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Release-store of a word to shared memory of a CTA of the cluster (a
+// shared::cluster address from mapa_shared).
+__device__ __forceinline__ void st_release_cluster_u32(uint32_t cluster_addr, uint32_t v)
+{
+    asm volatile("st.release.cluster.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
+// Acquire-load (cluster scope) of a word of this CTA's shared memory.
+__device__ __forceinline__ uint32_t ld_acquire_cluster_u32(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.acquire.cluster.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
 }
 
 __device__ __forceinline__ void cluster_sync_all()

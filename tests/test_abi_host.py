@@ -96,9 +96,10 @@ def test_kv_rejects(q):
     assert kv(A16, A16, 1, 4, 0, 128, A16, A16, A16, A16, A16, None) == 1
     assert kv(A16, A16, 0, 4, 8, 128, None, None, None, None, None, None) == 0
     sc = q.lib.quarot_kv_decode_scores
-    assert sc(A16, 1, 12, A16, A16, A16, 16, 8, 128, A16, None) == 2     # Hq % Hkv != 0
-    assert sc(A16, 1, 64 * 8, A16, A16, A16, 16, 8, 128, A16, None) == 2  # group of 64
-    assert sc(A16, 1, 64, A16, A16, A16, 0, 8, 128, None, None) == 0
+    assert sc(A16, 12, A16, A16, A16, 1, 16, 8, 128, A16, None) == 2     # Hq % Hkv != 0
+    assert sc(A16, 64 * 8, A16, A16, A16, 1, 16, 8, 128, A16, None) == 2  # group of 64
+    assert sc(A16, 64, A16, A16, A16, 1, 16, 8, 64, A16, None) == 2      # D != 128
+    assert sc(A16, 64, A16, A16, A16, 1, 0, 8, 128, None, None) == 0     # no tokens: no launch
     at = q.lib.quarot_kv_decode_attend
     assert at(A16, 1, 64, A16, A16, 16, 8, 64, A16, None) == 2       # D != 128
     assert at(A16, 1, 12, A16, A16, 16, 8, 128, A16, None) == 2      # Hq % Hkv != 0
@@ -155,3 +156,21 @@ def test_int8_entry_points_reject(q):
     need = ws(16, 256)
     assert f(A16, 16, 256, A16, 0, A16, A16, 256, A16, need - 1, A16, None) == 1
     assert f(A16, 16, 256, A16, 0, A16, A16, 256, P(0x10010), need, A16, None) == 3
+
+
+def test_timeout_entry_rejects(q):
+    A = ctypes.c_void_p(0x10000)
+    f = q.lib.quarot_test_wait_timeout
+    assert f(A, 0, A, A, 0, 1_000_000, None) == 1             # no rows
+    assert f(A, 256, A, A, 2, 1_000_000, None) == 1           # tile 2 of 2
+    assert f(A, 256, A, A, -1, 1_000_000, None) == 1
+    assert f(A, 256, A, A, 0, 10, None) == 1                  # limit too short
+    assert f(A, 256, A, A, 0, 3_000_000_000, None) == 1       # limit too long
+    assert f(ctypes.c_void_p(0x10008), 256, A, A, 0, 1_000_000, None) == 3
+
+
+def test_mma_probe_rejects(q):
+    n = ctypes.c_int64(0)
+    assert q.lib.quarot_probe_mma_i8(0, ctypes.byref(n), None) == 1
+    assert q.lib.quarot_probe_mma_i8((1 << 22) + 1, ctypes.byref(n), None) == 1
+    assert q.lib.quarot_probe_mma_i8(10, None, None) == 1

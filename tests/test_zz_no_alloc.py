@@ -9,11 +9,9 @@ run every other test already.
 """
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
-from parity import check_f16_output
 from rotation_bit_quantization_randomized_b200 import synth
 
 
@@ -46,7 +44,27 @@ def test_noalloc_matches_allocating_entry_on_two_calls(q):
         assert _noalloc(q, x, s, qw, sw, w.had_block, w.group, out, stream) == 0
         torch.cuda.synchronize()
         assert q.quarot_get_device_status() == 0
-        check_f16_output(out.cpu().numpy(), ref.cpu().numpy().astype(np.float64))
+        # the same kernels on the same inputs: the same bytes
+        assert torch.equal(out, ref)
+
+
+@pytest.mark.gpu
+def test_noalloc_at_the_scratch_limit(q):
+    # 4092 tokens x K 8192 with per-token scales need exactly 16 MiB: accepted
+    stream = torch.cuda.current_stream().cuda_stream
+    w = synth.LLAMA2_70B
+    M, N = 4092, 256
+    assert q.quarot_rotate_quant_linear_workspace(M, w.K, 0) == 16 * 1024 * 1024
+    x = torch.from_numpy(synth.activations(w, rows=M)).cuda()
+    W = torch.from_numpy(synth.weights(w, N)).cuda()
+    s = torch.from_numpy(synth.signs(w.K, w.seed)).cuda()
+    qw, sw = q.quarot_rotate_quant(W, s, 0, 0)
+    ref = q.quarot_rotate_quant_linear(x, s, qw, sw, 0, 0)
+    out = torch.full_like(ref, float("nan"))
+    assert _noalloc(q, x, s, qw, sw, 0, 0, out, stream) == 0
+    torch.cuda.synchronize()
+    assert q.quarot_get_device_status() == 0
+    assert torch.equal(out, ref)
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(q):
@@ -54,4 +72,6 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(q):
     # 8192 tokens x K 8192 need 32 MiB + scales > 16 MiB: rejected before any device work
     assert q.lib.quarot_rotate_quant_linear_noalloc(A, 8192, 8192, A, 0, 0, A, A, 256, A, None) == 2
     assert "16777216" in q.lib.quarot_last_error().decode()
+    # one token past the limit (4093 x K 8192: 16 MiB + 4 KiB) is rejected too
+    assert q.lib.quarot_rotate_quant_linear_noalloc(A, 4093, 8192, A, 0, 0, A, A, 256, A, None) == 2
     assert q.lib.quarot_rotate_quant_linear_noalloc(A, 0, 8192, A, 0, 0, A, A, 256, A, None) == 0
