@@ -67,6 +67,8 @@ def peaks():
 KERNEL_SOURCES = {
     "int4_gemm_pair_kernel": ["int4_gemm_pair.cuh", "int4_gemm.cuh", "tc_ptx.cuh", "common.cuh"],
     "fwht_quant_kernel": ["rotate_quant.cuh", "tc_ptx.cuh", "common.cuh"],
+    "had_tc_quant_kernel": ["rotate_tc.cuh", "rotate_quant.cuh", "kron_quant.cuh", "int4_gemm.cuh", "tc_ptx.cuh",
+                            "common.cuh"],
     "kv_quant_tma_kernel_keys": ["kv_quant.cuh", "rotate_quant.cuh", "tc_ptx.cuh", "common.cuh"],
     "kv_scores_kernel": ["kv_scores.cuh", "common.cuh"],
     "kv_attend_kernel": ["kv_attend.cuh", "common.cuh"],
@@ -421,9 +423,9 @@ def run_ours(args, rank, world, local_rank, dist):
                          "frac_of_nominal_4500": gemm_tops / 4500.0,
                          "frac_of_2x_bf16_burst": gemm_tops / (2.0 * pk["bf16"]),
                          "unit_note": "tera integer ops (2 per multiply-add), reported in the TFLOP/s field"},
-            "rotate_quant_roofline": {"bound": "hbm", "kernel": "fwht_quant_kernel<13,0,4> (quarot_rotate_quant)",
+            "rotate_quant_roofline": {"bound": "hbm", "kernel": "had_tc_quant_kernel<6,0,4> (quarot_rotate_quant)",
                                       "achieved": rq_gbs, "peak": pk["hbm"], "unit": "GB/s",
-                                      "frac": rq_gbs / pk["hbm"], "traffic": recorded_traffic("fwht_quant_kernel"),
+                                      "frac": rq_gbs / pk["hbm"], "traffic": recorded_traffic("had_tc_quant_kernel"),
                                       "peak_note": f"HBM copy {pk['src']}"},
             "components_ms": {"rotate_quant": k_ms[0], "int4_linear": k_ms[1], "kv_quant": k_ms[2],
                               "kv_decode_scores": k_ms[3]},

@@ -151,6 +151,27 @@ __device__ __forceinline__ float max3f(float a, float b, float c)
     return r;
 }
 
+// max |v[i]| over 128 values as a tree of three-input maxima (depth 5, not a
+// 64-long dependent chain).
+__device__ __forceinline__ float absmax128(const float (&v)[128])
+{
+    float a[43];
+#pragma unroll
+    for (int j = 0; j < 42; ++j)
+        a[j] = max3f(fabsf(v[3 * j]), fabsf(v[3 * j + 1]), fabsf(v[3 * j + 2]));
+    a[42] = fmaxf(fabsf(v[126]), fabsf(v[127]));
+    float b[15];
+#pragma unroll
+    for (int j = 0; j < 14; ++j)
+        b[j] = max3f(a[3 * j], a[3 * j + 1], a[3 * j + 2]);
+    b[14] = a[42];
+    float c[5];
+#pragma unroll
+    for (int j = 0; j < 5; ++j)
+        c[j] = max3f(b[3 * j], b[3 * j + 1], b[3 * j + 2]);
+    return max3f(max3f(c[0], c[1], c[2]), c[3], c[4]);
+}
+
 // (d0, d1) = (a0 * b + c, a1 * b + c) with one packed fp32x2 fused multiply-add.
 __device__ __forceinline__ void fma_x2(float a0, float a1, float b, float c, float &d0, float &d1)
 {

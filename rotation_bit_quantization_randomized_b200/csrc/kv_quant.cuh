@@ -125,17 +125,14 @@ kv_quant_tma_kernel(const __grid_constant__ CUtensorMap tmap,   // fp16 [rows, 1
         }
         if (ROTATE)
             fwht_bits<0, 7>(v);
-        float amax = 0.f;
-#pragma unroll
-        for (int k = 0; k < 128; k += 2)
-            amax = max3f(amax, fabsf(v[k]), fabsf(v[k + 1]));
+        const float amax = absmax128(v);
         const int64_t row = tile * kKvTileRows + t;
         const bool valid = row < rows;
         __half s16;
         const float r = group_scale(amax, scale_mul, sqrt_n, s16);
         if (valid)
             scales[row] = s16;
-        quant_pack_store<128>(v, r, q + (valid ? row : 0) * 64, valid);
+        quant_pack_store<128>(v, r, q + (valid ? row : 0) * 64, valid, scale_needs_clamp(s16));
     }
     // copies issued beyond the consumed tiles (abort only) land before exit:
     // iterations it .. issued - 1 had their copies issued but were not waited for

@@ -13,6 +13,7 @@
 #include "kv_scores.cuh"
 #include "mma_peak.cuh"
 #include "rotate_quant.cuh"
+#include "rotate_tc.cuh"
 
 #include <cuda.h>
 
@@ -150,6 +151,10 @@ quarot_status_t check_rotate_args(const void *x, int64_t M, int64_t K, const int
     return QUAROT_OK;
 }
 
+// Smallest log2 K of the full transform that takes the tensor-core kernel
+// (below it the register-only kernel).
+constexpr int kTcMinLogK = 8;
+
 // qmax of a code width: the largest code magnitude of the symmetric RTN.
 constexpr double qmax_of(int bits) { return (double)code_qmax(bits); }
 
@@ -203,6 +208,65 @@ quarot_status_t dispatch_fwht_asym(int logn, const void *x, int64_t M, const int
     }
 }
 
+quarot_status_t encode_tiled_fn_checked(void *&fn);
+
+// The full transform with its H_m factor on the tensor cores (K = 128 m).
+template <int LOGM, int GROUP, int BITS>
+quarot_status_t launch_had_tc(const void *x, int64_t M, const int8_t *signs, uint8_t *q, void *scales,
+                              cudaStream_t st, int dev, int sms)
+{
+    constexpr int m = 1 << LOGM;
+    constexpr int G = 256 / m;
+    if (M > ((int64_t(1) << 31) - 512) / m)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "M * K / 128 must stay below 2^31");
+    auto kern = had_tc_quant_kernel<LOGM, GROUP, BITS>;
+    int per_sm = 0;
+    quarot_status_t s = kernel_occupancy(kern, dev, kRtThreads, RtSmem::kBytes, per_sm);
+    if (s != QUAROT_OK)
+        return s;
+    void *fnp = nullptr;
+    s = encode_tiled_fn_checked(fnp);
+    if (s != QUAROT_OK)
+        return s;
+    auto fn = reinterpret_cast<CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                            const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                            const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                            CUtensorMapL2promotion, CUtensorMapFloatOOBfill)>(fnp);
+    // x viewed as fp16 [M * m, 128]: row (token, a), column b
+    CUtensorMap map;
+    const cuuint64_t dims[2] = {128, (cuuint64_t)M * m};
+    const cuuint64_t strides[1] = {256};
+    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(x), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(QUAROT_ERR_CUDA, "cuTensorMapEncodeTiled failed (code " + std::to_string((int)r) + ")");
+    const int64_t groups = (M + G - 1) / G;
+    const int grid = (int)std::min<int64_t>(groups, (int64_t)sms * per_sm);
+    const double n = double(128 * m);
+    kern<<<grid, kRtThreads, RtSmem::kBytes, st>>>(map, M, signs, q, scales,
+                                                   (float)(1.0 / (code_qmax(BITS) * std::sqrt(n))),
+                                                   (float)std::sqrt(n));
+    return after_launch("had_tc_quant_kernel launch");
+}
+
+template <int GROUP, int BITS>
+quarot_status_t dispatch_had_tc(int logn, const void *x, int64_t M, const int8_t *signs, uint8_t *q, void *scales,
+                                cudaStream_t st, int dev, int sms)
+{
+    switch (logn) {
+    case 8: return launch_had_tc<1, GROUP, BITS>(x, M, signs, q, scales, st, dev, sms);
+    case 9: return launch_had_tc<2, GROUP, BITS>(x, M, signs, q, scales, st, dev, sms);
+    case 10: return launch_had_tc<3, GROUP, BITS>(x, M, signs, q, scales, st, dev, sms);
+    case 11: return launch_had_tc<4, GROUP, BITS>(x, M, signs, q, scales, st, dev, sms);
+    case 12: return launch_had_tc<5, GROUP, BITS>(x, M, signs, q, scales, st, dev, sms);
+    case 13: return launch_had_tc<6, GROUP, BITS>(x, M, signs, q, scales, st, dev, sms);
+    default: return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "unsupported transform size");
+    }
+}
+
 template <bool ROTATE, int GROUP, int BITS = 4>
 quarot_status_t launch_block(const void *x, int64_t M, int64_t K, const int8_t *signs, uint8_t *q,
                              void *scales, float scale_mul, float sqrt_n, cudaStream_t st, int dev, int sms)
@@ -236,6 +300,15 @@ quarot_status_t rotate_quant_launch(const void *x, int64_t M, int64_t K, const i
     const int sms = info->sm_count;
     if (had_block == 0 && K >= 256) {
         const int logn = ilog2(K);
+        if (logn >= kTcMinLogK) {
+            // first factor H_{K/128} on the tensor cores, H_128 in registers
+            if (bits == 8)
+                return dispatch_had_tc<0, 8>(logn, x, M, signs, q, scales, st, dev, sms);
+            if (bits == 6)
+                return dispatch_had_tc<0, 6>(logn, x, M, signs, q, scales, st, dev, sms);
+            return group == 0 ? dispatch_had_tc<0, 4>(logn, x, M, signs, q, scales, st, dev, sms)
+                              : dispatch_had_tc<128, 4>(logn, x, M, signs, q, scales, st, dev, sms);
+        }
         if (bits == 8)
             return dispatch_fwht<0, 8>(logn, x, M, signs, q, scales, st, dev, sms);
         if (bits == 6)
@@ -296,6 +369,14 @@ quarot_status_t encode_tiled_fn(EncodeTiledFn &fn)
     }
     fn = cached;
     return QUAROT_OK;
+}
+
+quarot_status_t encode_tiled_fn_checked(void *&fn)
+{
+    EncodeTiledFn f;
+    quarot_status_t s = encode_tiled_fn(f);
+    fn = reinterpret_cast<void *>(f);
+    return s;
 }
 
 // Tensor map of a packed INT4 matrix [rows, K/2] bytes read in boxes of

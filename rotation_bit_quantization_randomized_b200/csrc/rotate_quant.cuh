@@ -50,16 +50,18 @@ constexpr int kBlockThreads = 128;
 // Quantizes 128 values of one thread and stores the 64 packed bytes.
 //  GROUP == 0: r = 7 / max|y| of the row; |v r| <= 7 (1 + 2^-23) so the
 //              rounding never leaves [-7, 7] and no clamp is needed.
-//  GROUP != 0: r = 1 / (sqrt(n) * fp16 scale); the clamp matters only when
-//              the fp16 scale is subnormal.
+//  GROUP != 0: r = 1 / (sqrt(n) * fp16 scale); with a normal fp16 scale
+//              |v r| <= 7 (1 + 2^-10) as well, so the clamp is needed (and
+//              taken, `clamp`) only when the fp16 scale is subnormal.
 template <int GROUP>
-__device__ __forceinline__ void quant_pack_store(const float (&v)[128], float r, uint8_t *dst, bool valid)
+__device__ __forceinline__ void quant_pack_store(const float (&v)[128], float r, uint8_t *dst, bool valid,
+                                                 bool clamp = true)
 {
     uint32_t pk[16];
 #pragma unroll
     for (int g = 0; g < 16; ++g) {
         uint32_t acc = 0;
-        if (GROUP == 0) {
+        if (GROUP == 0 || !clamp) {
             // two codes per packed fma: rint(t r) lands in the low mantissa bits
 #pragma unroll
             for (int k = 0; k < 8; k += 2) {
@@ -159,6 +161,14 @@ __device__ __forceinline__ float group_scale(float amax, float scale_mul, float 
     s16 = __float2half_rn(amax * scale_mul);
     const float sf = __half2float(s16);
     return (sf > 0.f && sf <= 65504.f) ? 1.0f / (sf * sqrt_n) : 0.f;
+}
+
+// Whether the codes under fp16 scale s16 can leave [-7, 7]: only a nonzero
+// subnormal scale rounds far enough below max|y| / 7.
+__device__ __forceinline__ bool scale_needs_clamp(__half s16)
+{
+    const unsigned short b = __half_as_ushort(s16);
+    return (b & 0x7C00u) == 0 && (b & 0x03FFu) != 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -484,15 +494,12 @@ block128_quant_kernel(const uint4 *__restrict__ x,     // [M, K] fp16, 8 per uin
                 block_signs(i, sg);
                 float v[128];
                 load_block<ROTATE>(xrow + (ok ? b : 0) * 16, ok, sg, v);
-                float amax = 0.f;
-#pragma unroll
-                for (int k = 0; k < 128; k += 2)
-                    amax = max3f(amax, fabsf(v[k]), fabsf(v[k + 1]));
+                const float amax = absmax128(v);
                 __half s16;
                 const float r = group_scale(amax, scale_mul, sqrt_n, s16);
                 if (ok)
                     reinterpret_cast<__half *>(scales)[row * nb + b] = s16;
-                quant_pack_store<GROUP>(v, r, qrow + (ok ? b : 0) * 64, ok);
+                quant_pack_store<GROUP>(v, r, qrow + (ok ? b : 0) * 64, ok, scale_needs_clamp(s16));
             }
         } else {
             // one scale per row: reduce the row maximum over the row's threads
