@@ -48,7 +48,7 @@ def parse():
     p.add_argument("--cpu-rows", type=int, default=2048, help="token rows of the CPU-baseline sample")
     p.add_argument("--case", choices=["gemm", "gemm_group", "gemm8", "gemm8_full", "gemm_asym", "rotate",
                                       "rotate_asym", "block", "kron", "kron_tok", "kvquant", "kvscores",
-                                      "kvattend", "kvattend_b64", "i8peak"],
+                                      "kvattend", "kvattend_b64", "kvdecode", "kvdecode_b64", "i8peak"],
                    default=None, help="time one kernel on a capture-sized workload (for ncu), not the step")
     return p.parse_args()
 
@@ -179,6 +179,11 @@ def bytes_kv_quant(B, T, H, D):
 
 def bytes_kv_scores(B, T, H, D, Hq):
     return B * T * H * (D // 2 + 2) + B * Hq * D * 2 + B * Hq * T * 4
+
+
+def bytes_kv_decode(B, T, H, D, Hq):
+    """The fused step: key and value codes + fp16 scales in, fp16 queries in, fp32 outputs out."""
+    return 2 * B * T * H * (D // 2 + 2) + B * Hq * D * 2 + B * Hq * D * 4
 
 
 def bytes_kv_attend(B, T, H, D, Hq):
@@ -516,7 +521,7 @@ def run_case(args):
         fn = lambda: q.quarot_rotate_quant(x, s, hb, group, qa, sa)
         work, unit = bytes_rotate_quant(M, K) / 1e9, "GB/s"
     else:
-        B, T, H, D, Hq = (64 if args.case == "kvattend_b64" else 16), 2048, 8, 128, 64
+        B, T, H, D, Hq = (64 if args.case in ("kvattend_b64", "kvdecode_b64") else 16), 2048, 8, 128, 64
         k = torch.randn((B, T, H, D), device=dev, generator=g).half()
         v = torch.randn((B, T, H, D), device=dev, generator=g).half()
         qh = torch.randn((B, Hq, D), device=dev, generator=g).half()
@@ -529,6 +534,10 @@ def run_case(args):
         elif args.case == "kvscores":
             fn = lambda: q.quarot_kv_decode_scores(qh, s, kq, ks, scores)
             work = bytes_kv_scores(B, T, H, D, Hq) / 1e9
+        elif args.case in ("kvdecode", "kvdecode_b64"):
+            o = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+            fn = lambda: q.quarot_kv_decode_attention(qh, s, kq, ks, vq, vs, o)
+            work = bytes_kv_decode(B, T, H, D, Hq) / 1e9
         else:
             q.quarot_kv_decode_scores(qh, s, kq, ks, scores)
             o = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)

@@ -435,6 +435,32 @@ quarot_status_t quarot_kv_decode_attend(const float *scores, int64_t B, int64_t 
                                         quarot_stream_t stream);
 
 /*
+ * quarot_kv_decode_attention -- one whole decode step of attention over the
+ * INT4 KV cache in one fused kernel [QR-A: the KV cache in 4 bits, the
+ * rotation covering aspects of the attention mechanism; DQ-12: a fixed
+ * Hadamard on the query-key product, per-head quantization, the attention
+ * output x value product on quantized values]:
+ *
+ *   q'[b,hq,:]  = (q[b,hq,:] * diag(signs[h,:])) * H_D / sqrt(D)   (fp32, h = hq / (Hq/Hkv))
+ *   s[b,hq,t]   = sum_d q'[d] * kq[b,t,h,d] * ks[b,t,h]
+ *   p[b,hq,t]   = softmax over t of s[b,hq,t] / sqrt(D)
+ *   out[b,hq,d] = sum_t p[b,hq,t] * vs[b,t,h] * vq[b,t,h,d]
+ *
+ * i.e. quarot_kv_decode_attend(quarot_kv_decode_scores(...)) without the
+ * scores in memory: the key and value codes are read once.  Both contractions
+ * run on the tensor cores with exact operands (codes in fp16; the fp32 query
+ * and softmax weights as two fp16 parts each) and fp32 accumulation.
+ * q_f16 [B, Hq, D] fp16; signs [Hkv, D] int8; kq, vq [B, T, Hkv, D/2] packed
+ * codes and ks_f16, vs_f16 [B, T, Hkv] fp16 scales (from quarot_kv_quant);
+ * out [B, Hq, D] fp32.  Limits: D == 128; T >= 1; Hq / Hkv in {1, 2, 4, 8,
+ * 16}; B, Hkv <= 65535.  B == 0 launches nothing.
+ */
+quarot_status_t quarot_kv_decode_attention(const void *q_f16, int64_t Hq, const int8_t *signs,
+                                           const uint8_t *kq, const void *ks_f16, const uint8_t *vq,
+                                           const void *vs_f16, int64_t B, int64_t T, int64_t Hkv,
+                                           int64_t D, float *out, quarot_stream_t stream);
+
+/*
  * quarot_get_device_status -- synchronizes `stream` (the whole current device
  * when stream is NULL), then reports (and clears) the library's device-side
  * error word: QUAROT_ERR_DEVICE_TIMEOUT if any kernel since the last call

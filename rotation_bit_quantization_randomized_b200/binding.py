@@ -50,6 +50,7 @@ _SIGS = {
     "quarot_rotate_quant_kron": ([_P, _I64, _I64, _P, _I64, _P, _P, _P], _INT),
     "quarot_kron_factor": ([_I64, _P], _INT),
     "quarot_kv_decode_attend": ([_P, _I64, _I64, _P, _P, _I64, _I64, _I64, _P, _P], _INT),
+    "quarot_kv_decode_attention": ([_P, _I64, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P], _INT),
     "quarot_probe_mma_i8": ([_I64, _P, _P], _INT),
     "quarot_test_wait_timeout": ([_P, _I64, _P, _P, _I64, ctypes.c_uint64, _P], _INT),
     "quarot_get_device_status": ([_P], _INT),
@@ -375,6 +376,20 @@ def quarot_kv_decode_attend(scores: torch.Tensor, vq: torch.Tensor, vs: torch.Te
     _check("quarot_kv_decode_attend",
            lib.quarot_kv_decode_attend(_ptr(scores), B, Hq, _ptr(vq), _ptr(vs), T, Hkv, 128, _ptr(out),
                                        _stream(stream)))
+    return out
+
+
+def quarot_kv_decode_attention(q: torch.Tensor, signs: torch.Tensor, kq: torch.Tensor, ks: torch.Tensor,
+                               vq: torch.Tensor, vs: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None):
+    """One fused decode step: q fp16 [B, Hq, 128] against the INT4 K and V caches
+    [B, T, Hkv, 64] (+ fp16 scales [B, T, Hkv]) -> fp32 [B, Hq, 128]."""
+    B, Hq, D = q.shape
+    _, T, H, _ = kq.shape
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
+    _check("quarot_kv_decode_attention",
+           lib.quarot_kv_decode_attention(_ptr(q), Hq, _ptr(signs), _ptr(kq), _ptr(ks), _ptr(vq), _ptr(vs), B, T, H,
+                                          D, _ptr(out), _stream(stream)))
     return out
 
 

@@ -1,0 +1,565 @@
+// kv_decode_tc.cuh -- one fused decode step of attention over the INT4 KV
+// cache on the tensor cores: the query rotation, the query-key scores, the
+// softmax and the product with the value cache in one kernel, so that the
+// key and value codes are read once and the scores never reach global memory
+// (QuaRot abstract: the KV cache in 4 bits and the rotation applied to
+// aspects of the attention mechanism; DuQuant Knowl 12: a fixed Hadamard on
+// the query-key product, per-head quantization, the softmax output times the
+// quantized values; QuaRot summary, References: FlashInfer):
+//
+//   q'[g]      = (q[g] * diag(s_h)) H_128 / sqrt(128)                (fp32)
+//   s[g, t]    = ks[t] * sum_d q'[g, d] kcode[t, d]
+//   p[g, t]    = softmax over t of s[g, t] / sqrt(128)
+//   out[g, d]  = sum_t p[g, t] vs[t] vcode[t, d]
+//
+// for the G query heads g of one KV head h.  Both contractions run as
+// tcgen05.mma kind::f16 with fp32 accumulation in tensor memory, on exact
+// operands: the codes are small integers (exact in fp16), and the fp32 query
+// and weights are split into two fp16 rows each, hi = fp16(x 2^e) and lo =
+// fp16((x 2^e - hi) 2^11), with a per-head power of two e, so that hi + lo
+// 2^-11 carries 22 bits of x and every product with a code is exact:
+//   scores:  D_s[t][n] = sum_p A_k[t][p] B_q[n][p]    (M 128 tokens, N rows n of B_q, K 128)
+//   values:  D_o[p][n] = sum_t A_v[p][t] B_w[n][t]    (M 128 dims, N rows n of B_w, K 128 tokens)
+// where row n < G of B is head n's hi part and row G + n its lo part (rows
+// past 2 G, when G < 8, only feed accumulator columns that are never read).  A_k
+// (key codes, K-major) and A_v (value codes, MN-major: the dims of a token
+// are contiguous) share one 128 x 128 fp16 tile layout in shared memory, so
+// one conversion routine serves both; it emits the dims of every group of
+// four in the order (0, 2, 1, 3) (two nibble bytes become a low-nibble and a
+// high-nibble half2 word), and the query rows use the same order, so each dot
+// product is unchanged and output lane p holds dim d(p).
+//
+// A cluster of S CTAs covers one (batch, KV head); CTA r walks its slice of
+// the tokens in tiles of 128 with the running-maximum softmax (in base 2: the
+// scores carry the factor log2(e) / sqrt(128) and the exponentials are exp2):
+// per tile the key codes are converted and multiplied, the 128 threads (one
+// per token) read their scores, the tile maximum updates the running maximum
+// m and the sum l, the value accumulator D_o is rescaled in tensor memory when
+// m grows, the weights e * vs (one power-of-two scale for the whole slice,
+// from its largest value scale) are written as B_w, and the value codes
+// (converted into the same tile) are multiplied into D_o.  The next
+// tile's codes arrive by asynchronous copies meanwhile.  At the end the CTAs
+// of the cluster combine their (m, l, acc) through distributed shared memory:
+// out = sum_r exp(m_r - M) acc_r / sum_r exp(m_r - M) l_r, M = max_r m_r.
+// Several CTAs share an SM (about 60 KB of shared memory and 32 or 64
+// tensor-memory columns each), so one CTA's conversions overlap another's
+// waits.  Every wait is bounded.
+#pragma once
+
+#include "common.cuh"
+#include "kron_quant.cuh"
+#include "kv_attend.cuh"
+#include "tc_ptx.cuh"
+
+namespace quarot {
+
+constexpr int kDecThreads = 128;
+constexpr int kDecTile = 128;                    // tokens per tile
+constexpr int kDecMaxSplit = 8;
+constexpr uint64_t kDecWaitLimitNs = 2000000000ull;
+
+template <int G>
+struct DecShape {
+    static constexpr int NP = G <= 8 ? 16 : 32;            // MMA N: G hi rows, G lo rows, zero padding
+    static constexpr int kTmemCols = G <= 8 ? 32 : 64;     // D_s at column 0, D_o at column NP
+    static constexpr int kTileOff = 0;                     // code tile: 2 panels of 128 rows x 128 B
+    static constexpr int kBqOff = 32768;                   // B_q: 2 panels of NP rows x 128 B
+    static constexpr int kBwOff = kBqOff + 2 * NP * 128;   // B_w: the same shape
+    static constexpr int kStageBytes = 2 * kDecTile * 64;  // raw codes of one tile: K then V, 64 B a token
+    static constexpr int kStageOff = kBwOff + 2 * NP * 128; // two stages: tiles j + 1 and j + 2 in flight
+    static constexpr int kMiscOff = kStageOff + 2 * kStageBytes;
+    // misc: mbarrier (8), tmem slot (4), pad (4), drain mbarrier (8), pad, then floats:
+    //   red[4][G + 1]  per-warp tile maxima of each head's scores
+    //   m[G], l[G], lpart[4][G], inv_qs[G], vmx[4]
+    static constexpr int kRedOff = kMiscOff + 32;
+    static constexpr int kQmaxOff = kRedOff + 4 * (G + 1) * 4;
+    static constexpr int kMOff = kQmaxOff + 4 * G * 4;
+    static constexpr int kLOff = kMOff + G * 4;
+    static constexpr int kLpOff = kLOff + G * 4;
+    static constexpr int kIqOff = kLpOff + 4 * G * 4;       // 1 / 2^e of each head's query
+    static constexpr int kVmOff = kIqOff + G * 4;           // per-warp maxima of the slice's value scales
+    static constexpr int kBytes = kVmOff + 16 + 1024;
+    // the code tile is free after the last tile: the CTA's unnormalized
+    // result fin[G][128] fp32 lives there then
+    static constexpr int kFinOff = kTileOff;
+    static_assert(kBqOff % 1024 == 0 && kBwOff % 1024 == 0 && kStageOff % 16 == 0, "alignment");
+};
+
+// dim held by position p of a converted row: (0, 2, 1, 3) within each group of four
+__host__ __device__ constexpr int dec_dim(int p) { return (p & ~3) | ((p & 1) << 1) | ((p >> 1) & 1); }
+
+// Converts one token's 64 bytes of packed codes (four uint4) into its row of
+// the fp16 tile (row t; 128-byte-swizzled chunks in two 64-column panels).
+// Bytes j, j + 1 -> x = b_j | b_{j+1} << 16 (biased by XOR 0x88: u = c + 8);
+// low nibbles: half2 (0x6400 | u) - 1032 = c; high nibbles: half2 (0x6400 |
+// 16 u) * 1/16 - 72 = c; both exact.
+__device__ __forceinline__ void dec_convert_row(const uint4 (&w)[4], uint8_t *tile, int t)
+{
+    const __half2 kSub = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));   // 1032
+    const __half2 kMul = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));   // 1/16
+    const __half2 kOff = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));   // -72
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {                      // 16-byte output chunk c: dims 8c .. 8c + 7
+        const uint4 in = w[c >> 2];
+        const uint32_t word = ((c & 3) == 0 ? in.x : (c & 3) == 1 ? in.y : (c & 3) == 2 ? in.z : in.w) ^ 0x88888888u;
+        uint32_t o[4];
+#pragma unroll
+        for (int hpair = 0; hpair < 2; ++hpair) {
+            const uint32_t x = __byte_perm(word, 0u, hpair == 0 ? 0x4140 : 0x4342);
+            const uint32_t lo = (x & 0x000F000Fu) | 0x64006400u;
+            const uint32_t hi = (x & 0x00F000F0u) | 0x64006400u;
+            __half2 hl, hh;
+            memcpy(&hl, &lo, 4);
+            memcpy(&hh, &hi, 4);
+            hl = __hsub2(hl, kSub);
+            hh = __hfma2(hh, kMul, kOff);
+            memcpy(&o[2 * hpair], &hl, 4);
+            memcpy(&o[2 * hpair + 1], &hh, 4);
+        }
+        const int panel = c >> 3, ch = c & 7;
+        *reinterpret_cast<uint4 *>(tile + panel * 16384 + t * 128 + ((ch ^ (t & 7)) << 4)) =
+            make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+// Writes x (fp32) as the hi / lo fp16 pair of rows n and n + G at column k of
+// a K-major B tile (two 64-column panels of NP rows x 128 B, 128-byte swizzle).
+template <int G>
+__device__ __forceinline__ void dec_put_split(uint8_t *b, int n, int k, float xs)
+{
+    constexpr int NP = DecShape<G>::NP;
+    const __half hi = __float2half_rn(xs);
+    const __half lo = __float2half_rn((xs - __half2float(hi)) * 2048.0f);
+    const int panel = k >> 6, kk = k & 63;
+    auto at = [&](int row) {
+        return reinterpret_cast<__half *>(b + panel * (NP * 128) + row * 128 + ((((kk >> 3) ^ (row & 7))) << 4)) +
+               (kk & 7);
+    };
+    *at(n) = hi;
+    *at(G + n) = lo;
+}
+
+// Power of two 2^e that brings max|x| (> 0) into [2^14, 2^15): hi parts then
+// stay far from fp16 overflow and lo parts keep 11 more bits.  Built from the
+// exponent bits, so 2^e and its inverse are exact; 1 for a zero maximum.
+__device__ __forceinline__ float dec_pow2_scale(float amax, float &inv)
+{
+    const int ex = (int)((__float_as_uint(amax) >> 23) & 0xFFu);     // biased exponent of amax
+    if (!(amax > 0.f) || ex == 0xFF) {
+        inv = 1.0f;
+        return 1.0f;
+    }
+    const int e = min(max(14 - (ex - 127), -126), 126);
+    inv = __uint_as_float((uint32_t)(127 - e) << 23);
+    return __uint_as_float((uint32_t)(127 + e) << 23);
+}
+
+template <int G>
+__global__ void __launch_bounds__(kDecThreads)
+kv_decode_tc_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
+                    const int8_t *__restrict__ signs,    // [Hkv, 128]
+                    const uint8_t *__restrict__ kq,      // [B, T, Hkv, 64 bytes]
+                    const __half *__restrict__ ks,       // [B, T, Hkv]
+                    const uint8_t *__restrict__ vq,      // [B, T, Hkv, 64 bytes]
+                    const __half *__restrict__ vs,       // [B, T, Hkv]
+                    int64_t T, int Hkv, float *__restrict__ out)   // [B, Hq, 128]
+{
+    using S = DecShape<G>;
+    constexpr int NP = S::NP;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *tile = smem + S::kTileOff;
+    uint8_t *bq = smem + S::kBqOff;
+    uint8_t *bw = smem + S::kBwOff;
+    uint8_t *stages = smem + S::kStageOff;
+    const uint32_t bar = smem_u32(smem + S::kMiscOff);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + S::kMiscOff + 8);
+    const uint32_t bar_drain = smem_u32(smem + S::kMiscOff + 16);
+    float *red = reinterpret_cast<float *>(smem + S::kRedOff);      // [4][G + 1]
+    float *sm_m = reinterpret_cast<float *>(smem + S::kMOff);
+    float *sm_l = reinterpret_cast<float *>(smem + S::kLOff);
+    float *lpart = reinterpret_cast<float *>(smem + S::kLpOff);     // [4][G]
+    float *fin = reinterpret_cast<float *>(smem + S::kFinOff);      // [G][128]
+    float *inv_qs = reinterpret_cast<float *>(smem + S::kIqOff);    // [G]
+    float *vmx = reinterpret_cast<float *>(smem + S::kVmOff);       // [4]
+
+    const int nsplit = gridDim.x;
+    const int r = blockIdx.x;
+    const int h = blockIdx.y;
+    const int64_t b = blockIdx.z;
+    const int Hq = Hkv * G;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const float kInvSqrtD = 0.08838834764831845f;
+    // softmax in base 2: scores / sqrt(128) times log2(e), then exp2
+    const float kScoreMul = 0.08838834764831845f * 1.4426950408889634f;
+    const int64_t slice = (T + nsplit - 1) / nsplit;
+    const int64_t ts = min(T, (int64_t)r * slice);
+    const int64_t te = min(T, ts + slice);
+    const int ntiles = (int)((te - ts + kDecTile - 1) / kDecTile);
+
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        mbar_init(bar_drain, 1);
+        mbar_fence_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tmem_slot), S::kTmemCols);
+        tmem_relinquish();
+    }
+    // raw codes of tile j into stage j % 2: thread t copies token t's key and
+    // value rows; every call commits one group (empty past the last tile), so
+    // that "all but the latest group done" always means "tile j has landed"
+    auto issue_copy = [&](int j) {
+        const int64_t t = ts + (int64_t)j * kDecTile + tid;
+        uint8_t *stage = stages + (j & 1) * S::kStageBytes;
+        const uint32_t dk = smem_u32(stage + tid * 64), dv = smem_u32(stage + kDecTile * 64 + tid * 64);
+        if (j < ntiles && t < te) {
+            const uint8_t *sk = kq + ((b * T + t) * Hkv + h) * 64;
+            const uint8_t *sv = vq + ((b * T + t) * Hkv + h) * 64;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                cp_async16(dk + 16 * c, sk + 16 * c);
+                cp_async16(dv + 16 * c, sv + 16 * c);
+            }
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    issue_copy(0);
+    issue_copy(1);
+
+    // ---- the slice's largest value scale (the weights e * vs never exceed
+    // it, so one power-of-two scale serves every tile of the slice)
+    {
+        float vm = 0.f;
+        for (int j = 0; j < ntiles; ++j) {
+            const int64_t t = ts + (int64_t)j * kDecTile + tid;
+            if (t < te)
+                vm = fmaxf(vm, __half2float(vs[(b * T + t) * Hkv + h]));
+        }
+        vm = warp_max(vm, 32);
+        if (lane == 0)
+            vmx[warp] = vm;
+    }
+    // ---- rotate the G queries (16 threads per query, 8 elements each: bits
+    // 0-2 in registers, bits 3-6 through half-warp shuffles), as in the
+    // decode-scores kernel; the 16 threads of a query then find its maximum
+    // and write its hi / lo rows of B_q in the converted dim order
+    {
+        const int p = tid & 15;
+        const int8_t *sg = signs + h * 128 + 8 * p;
+#pragma unroll
+        for (int g0 = 0; g0 < G; g0 += kDecThreads / 16) {
+            const int g = g0 + (tid >> 4);
+            const bool gv = G % (kDecThreads / 16) == 0 || g < G;
+            const uint4 raw = gv ? *reinterpret_cast<const uint4 *>(q + (b * Hq + (int64_t)h * G + g) * 128 + 8 * p)
+                                 : make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+            float v[8];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float2 f = half2_bits_to_float2(w4[k]);
+                v[2 * k] = sg[2 * k] < 0 ? -f.x : f.x;
+                v[2 * k + 1] = sg[2 * k + 1] < 0 ? -f.y : f.y;
+            }
+#pragma unroll
+            for (int hb = 1; hb < 8; hb <<= 1)
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    if ((i & hb) == 0) {
+                        const float a = v[i], c = v[i + hb];
+                        v[i] = a + c;
+                        v[i + hb] = a - c;
+                    }
+#pragma unroll
+            for (int lb = 1; lb < 16; lb <<= 1) {
+                const bool upper = (p & lb) != 0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float o = __shfl_xor_sync(0xffffffffu, v[i], lb);
+                    v[i] = upper ? o - v[i] : v[i] + o;
+                }
+            }
+            float mx = 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                v[i] *= kInvSqrtD;
+                mx = fmaxf(mx, fabsf(v[i]));
+            }
+#pragma unroll
+            for (int lb = 1; lb < 16; lb <<= 1)
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, lb));
+            float inv;
+            const float sc = dec_pow2_scale(mx, inv);
+            if (gv) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    dec_put_split<G>(bq, g, 8 * p + dec_dim(i), v[i] * sc);
+                if (p == 0)
+                    inv_qs[g] = inv;
+            }
+        }
+    }
+    if (tid < G) {
+        sm_m[tid] = -INFINITY;
+        sm_l[tid] = 0.f;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    float inv_wsc;
+    const float wsc = dec_pow2_scale(fmaxf(fmaxf(vmx[0], vmx[1]), fmaxf(vmx[2], vmx[3])), inv_wsc);
+    float inv_q[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+        inv_q[g] = inv_qs[g];
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
+
+    float lsum[G];                                    // this thread's share of sum exp2
+    float m_run[G];                                   // running maximum (base-2 units)
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        lsum[g] = 0.f;
+        m_run[g] = -INFINITY;
+    }
+    uint32_t commits = 0;
+    bool ok = true;
+    constexpr uint32_t idesc_s = idesc_f16(128, NP);
+    constexpr uint32_t idesc_o = idesc_f16(128, NP) | (1u << 15);    // A (values) MN-major
+    auto mma_wait = [&]() {
+        // the latest commit has completed (bounded; the CTA then gives up as a whole)
+        bool done = true;
+        if (!mbar_try_wait(bar, (commits - 1) & 1)) {
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(bar, (commits - 1) & 1)) {
+                if (globaltimer_ns() - t0 > kDecWaitLimitNs) {
+                    record_timeout();
+                    done = false;
+                    break;
+                }
+            }
+        }
+        return __syncthreads_and(done) != 0;
+    };
+
+    // scales of token t of tile j (loaded one tile ahead)
+    auto load_scales = [&](int j, float &ksv, float &vsv) {
+        const int64_t t = ts + (int64_t)j * kDecTile + tid;
+        const bool tv = j < ntiles && t < te;
+        ksv = tv ? __half2float(ks[(b * T + t) * Hkv + h]) : 0.f;
+        vsv = tv ? __half2float(vs[(b * T + t) * Hkv + h]) : 0.f;
+    };
+    float ks_next, vs_next;
+    load_scales(0, ks_next, vs_next);
+#pragma unroll 1
+    for (int j = 0; j < ntiles && ok; ++j) {
+        const int64_t t = ts + (int64_t)j * kDecTile + tid;
+        const bool tv = t < te;
+        const float ksv = ks_next, vsv = vs_next;
+        load_scales(j + 1, ks_next, vs_next);
+        const uint8_t *stage = stages + (j & 1) * S::kStageBytes;
+        // the previous tile's value MMAs are done with the code tile
+        if (j > 0 && !(ok = mma_wait()))
+            break;
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+        __syncthreads();
+        // ---- keys: convert, multiply with the query rows
+        {
+            uint4 w[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                w[c] = tv ? *reinterpret_cast<const uint4 *>(stage + tid * 64 + 16 * c)
+                          : make_uint4(0u, 0u, 0u, 0u);
+            dec_convert_row(w, tile, tid);
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                umma_f16_ss(tmem, desc_kmajor_sw128(smem_u32(tile) + 16384 * (kk >> 2) + 32 * (kk & 3)),
+                            desc_kmajor_sw128(smem_u32(bq) + NP * 128 * (kk >> 2) + 32 * (kk & 3)), idesc_s,
+                            kk > 0 ? 1u : 0u);
+            umma_commit(bar);
+        }
+        ++commits;
+        if (!(ok = mma_wait()))
+            break;
+        tc_fence_after();
+        // ---- scores of token t (lane t of D_s), the tile maxima
+        float s[G];
+        {
+            uint32_t d[NP];
+            if constexpr (NP == 16) {
+                uint32_t (&d16)[16] = *reinterpret_cast<uint32_t (*)[16]>(d);
+                tmem_ld16(lane_base, d16);
+                tmem_wait_ld16(d16);
+            } else {
+                uint32_t (&d32)[32] = *reinterpret_cast<uint32_t (*)[32]>(d);
+                tmem_ld32(lane_base, d32);
+                tmem_wait_ld(d32);
+            }
+            // score / sqrt(128) in base-2 units: (hi + lo 2^-11) 2^-e ks / sqrt(128) log2(e)
+            const float km = ksv * kScoreMul;
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float x = (__uint_as_float(d[g]) + __uint_as_float(d[G + g]) * (1.0f / 2048.0f)) * inv_q[g];
+                s[g] = tv ? x * km : -INFINITY;
+            }
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float mg = warp_max(s[g], 32);
+            if (lane == 0)
+                red[warp * (G + 1) + g] = mg;
+        }
+        __syncthreads();
+        float beta[G];                               // rescale of the value accumulator
+        bool rescale = false;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float tmax = fmaxf(fmaxf(red[g], red[(G + 1) + g]), fmaxf(red[2 * (G + 1) + g], red[3 * (G + 1) + g]));
+            const float m_new = fmaxf(m_run[g], tmax);
+            const float alpha = m_run[g] == -INFINITY ? 0.f : exp2f(m_run[g] - m_new);
+            beta[g] = alpha;
+            rescale |= j > 0 && alpha != 1.0f;
+            const float e = tv ? exp2f(s[g] - m_new) : 0.f;
+            lsum[g] = lsum[g] * alpha + e;
+            m_run[g] = m_new;
+            dec_put_split<G>(bw, g, tid, e * vsv * wsc);
+        }
+        // the value accumulator in the units of this tile (lane = dim)
+        if (rescale) {
+            uint32_t d[NP];
+            if constexpr (NP == 16) {
+                uint32_t (&d16)[16] = *reinterpret_cast<uint32_t (*)[16]>(d);
+                tmem_ld16(lane_base + NP, d16);
+                tmem_wait_ld16(d16);
+            } else {
+                uint32_t (&d32)[32] = *reinterpret_cast<uint32_t (*)[32]>(d);
+                tmem_ld32(lane_base + NP, d32);
+                tmem_wait_ld(d32);
+            }
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                d[g] = __float_as_uint(__uint_as_float(d[g]) * beta[g]);
+                d[G + g] = __float_as_uint(__uint_as_float(d[G + g]) * beta[g]);
+            }
+            if constexpr (NP == 16)
+                tmem_st16(lane_base + NP, *reinterpret_cast<uint32_t (*)[16]>(d));
+            else
+                tmem_st32(lane_base + NP, *reinterpret_cast<uint32_t (*)[32]>(d));
+            tmem_wait_st();
+        }
+        // ---- values: convert into the same tile (the key MMAs are done)
+        {
+            uint4 w[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                w[c] = tv ? *reinterpret_cast<const uint4 *>(stage + kDecTile * 64 + tid * 64 + 16 * c)
+                          : make_uint4(0u, 0u, 0u, 0u);
+            dec_convert_row(w, tile, tid);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        // stage j % 2 is consumed: tile j + 2 may land there
+        issue_copy(j + 2);
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                umma_f16_ss(tmem + NP, desc_mnmajor_sw128(smem_u32(tile) + 2048 * kk, 16384),
+                            desc_kmajor_sw128(smem_u32(bw) + NP * 128 * (kk >> 2) + 32 * (kk & 3)), idesc_o,
+                            (j > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(bar);
+        }
+        ++commits;
+    }
+    if (ok && ntiles > 0)
+        ok = mma_wait();
+    asm volatile("cp.async.wait_all;" ::: "memory");
+
+    // ---- this CTA's partial result: fin[g][d] (unnormalized), m, l
+    if (ok && ntiles > 0) {
+        tc_fence_after();
+        uint32_t d[NP];
+        if constexpr (NP == 16) {
+            uint32_t (&d16)[16] = *reinterpret_cast<uint32_t (*)[16]>(d);
+            tmem_ld16(lane_base + NP, d16);
+            tmem_wait_ld16(d16);
+        } else {
+            uint32_t (&d32)[32] = *reinterpret_cast<uint32_t (*)[32]>(d);
+            tmem_ld32(lane_base + NP, d32);
+            tmem_wait_ld(d32);
+        }
+        const int dim = dec_dim(tid);
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+            fin[g * 128 + dim] = (__uint_as_float(d[g]) + __uint_as_float(d[G + g]) * (1.0f / 2048.0f)) * inv_wsc;
+    } else {
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+            fin[g * 128 + tid] = 0.f;
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        const float ls = warp_sum_f(lsum[g]);
+        if (lane == 0)
+            lpart[warp * G + g] = ls;
+    }
+    __syncthreads();
+    if (tid < G) {
+        sm_l[tid] = ntiles > 0 ? (lpart[tid] + lpart[G + tid]) + (lpart[2 * G + tid] + lpart[3 * G + tid]) : 0.f;
+        sm_m[tid] = ntiles > 0 ? m_run[tid] : -INFINITY;
+    }
+
+    // combine the slices of the cluster: CTA r finishes heads r, r + S, ...
+    cluster_sync_all();
+    const uint32_t a_fin = smem_u32(fin);
+    const uint32_t a_m = smem_u32(sm_m);
+    const uint32_t a_l = smem_u32(sm_l);
+    for (int g = r; g < G; g += nsplit) {
+        float mq[kDecMaxSplit], lq[kDecMaxSplit], fq[kDecMaxSplit];
+#pragma unroll
+        for (int qq = 0; qq < kDecMaxSplit; ++qq) {
+            if (qq < nsplit) {
+                mq[qq] = ld_dsmem_f32(mapa_shared(a_m + 4 * g, qq));
+                lq[qq] = ld_dsmem_f32(mapa_shared(a_l + 4 * g, qq));
+                fq[qq] = ld_dsmem_f32(mapa_shared(a_fin + 4 * (g * 128 + tid), qq));
+            } else {
+                mq[qq] = -INFINITY;
+                lq[qq] = 0.f;
+                fq[qq] = 0.f;
+            }
+        }
+        float M = -INFINITY;
+#pragma unroll
+        for (int qq = 0; qq < kDecMaxSplit; ++qq)
+            M = fmaxf(M, mq[qq]);
+        float num = 0.f, den = 0.f;
+#pragma unroll
+        for (int qq = 0; qq < kDecMaxSplit; ++qq) {
+            const float f = mq[qq] == -INFINITY ? 0.f : exp2f(mq[qq] - M);
+            den = fmaf(f, lq[qq], den);
+            num = fmaf(f, fq[qq], num);
+        }
+        out[(b * Hq + (int64_t)h * G + g) * 128 + tid] = num / den;
+    }
+    // every MMA this CTA issued has completed (also after a timeout)
+    if (tid == 0) {
+        umma_commit(bar_drain);
+        mbar_wait_drain(bar_drain, 0, kDecWaitLimitNs);
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();                   // no CTA leaves while another may still read its memory
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, S::kTmemCols);
+    }
+}
+
+}  // namespace quarot

@@ -9,6 +9,7 @@
 #include "int8_gemm_pair.cuh"
 #include "kron_quant.cuh"
 #include "kv_attend.cuh"
+#include "kv_decode_tc.cuh"
 #include "kv_quant.cuh"
 #include "kv_scores.cuh"
 #include "mma_peak.cuh"
@@ -806,6 +807,90 @@ quarot_status_t attend_resident_clusters(int G, int split, int dev, int &fit)
     return QUAROT_OK;
 }
 
+// Clusters of `split` fused decode CTAs (G query heads per KV head) that can
+// be resident at once, queried once per (device, G, split); also raises the
+// kernel's dynamic shared-memory limit.
+template <int G>
+quarot_status_t decode_resident_clusters(int split, int dev, int &fit)
+{
+    static int cache[kMaxDevices][4];
+    static bool known[kMaxDevices][4];
+    const int si = split == 1 ? 0 : split == 2 ? 1 : split == 4 ? 2 : 3;
+    {
+        std::lock_guard<std::mutex> lk(g_mutex);
+        if (known[dev][si]) {
+            fit = cache[dev][si];
+            return QUAROT_OK;
+        }
+    }
+    cudaError_t e = cudaFuncSetAttribute(kv_decode_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)DecShape<G>::kBytes);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaFuncSetAttribute");
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)split, 1, 1);
+    cfg.blockDim = dim3(kDecThreads);
+    cfg.dynamicSmemBytes = DecShape<G>::kBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)split;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaOccupancyMaxActiveClusters(&fit, kv_decode_tc_kernel<G>, &cfg);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaOccupancyMaxActiveClusters");
+    std::lock_guard<std::mutex> lk(g_mutex);
+    cache[dev][si] = fit;
+    known[dev][si] = true;
+    return QUAROT_OK;
+}
+
+template <int G>
+quarot_status_t launch_decode_tc(const __half *q, const int8_t *signs, const uint8_t *kq, const __half *ks,
+                                 const uint8_t *vq, const __half *vs, int64_t B, int64_t T, int Hkv, float *out,
+                                 cudaStream_t st, int dev)
+{
+    // tokens split over a cluster of S CTAs, at least 128 tokens each: the S
+    // whose B * Hkv * S CTAs fill the resident slots best, then the one with
+    // fewer waves
+    const int smax = T >= 1024 ? 8 : T >= 512 ? 4 : T >= 256 ? 2 : 1;
+    int split = smax;
+    double best_eff = -1.0;
+    int64_t best_waves = 0;
+    for (int sp = smax; sp >= 1; sp /= 2) {
+        int fit = 0;
+        quarot_status_t s = decode_resident_clusters<G>(sp, dev, fit);
+        if (s != QUAROT_OK)
+            return s;
+        const int64_t clusters = B * Hkv;
+        const int64_t waves = fit > 0 ? (clusters + fit - 1) / fit : clusters;
+        const double eff = fit > 0 ? (double)clusters / ((double)waves * fit) : 0.0;
+        if (eff > best_eff + 1e-9 || (eff > best_eff - 1e-9 && waves < best_waves)) {
+            best_eff = eff;
+            best_waves = waves;
+            split = sp;
+        }
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)split, (unsigned)Hkv, (unsigned)B);
+    cfg.blockDim = dim3(kDecThreads);
+    cfg.dynamicSmemBytes = DecShape<G>::kBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)split;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kv_decode_tc_kernel<G>, q, signs, kq, ks, vq, vs, T, Hkv, out);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "kv_decode_tc_kernel launch");
+    return after_launch("kv_decode_tc_kernel launch");
+}
+
 }  // namespace
 
 // Tensor map of an fp16 [rows, 128] matrix (KV rows of one head) read in
@@ -1374,6 +1459,47 @@ quarot_status_t quarot_test_wait_timeout(const void *v_f16, int64_t rows, uint8_
         return s;
     return launch_kv_tma<false>(v_f16, rows, 1, nullptr, q_packed, scales_f16, (float)(1.0 / 7.0), 1.0f,
                                 (cudaStream_t)stream, dev, info->sm_count, wait_limit_ns, withheld_tile);
+}
+
+quarot_status_t quarot_kv_decode_attention(const void *q_f16, int64_t Hq, const int8_t *signs, const uint8_t *kq,
+                                           const void *ks_f16, const uint8_t *vq, const void *vs_f16, int64_t B,
+                                           int64_t T, int64_t Hkv, int64_t D, float *out, quarot_stream_t stream)
+{
+    if (B < 0 || T <= 0 || Hkv <= 0 || Hq <= 0)
+        return fail(QUAROT_ERR_INVALID_ARG, "B must be >= 0; T, Hq, Hkv > 0");
+    if (D != 128)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "head dimension must be 128");
+    if (Hq % Hkv != 0)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "Hq must be a multiple of Hkv");
+    const int64_t G = Hq / Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "Hq / Hkv must be 1, 2, 4, 8 or 16");
+    if (Hkv > 65535 || B > 65535)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "B and Hkv must be <= 65535");
+    if (B == 0)
+        return QUAROT_OK;
+    if (!q_f16 || !signs || !kq || !ks_f16 || !vq || !vs_f16 || !out)
+        return fail(QUAROT_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(q_f16) || !aligned16(kq) || !aligned16(ks_f16) || !aligned16(vq) || !aligned16(vs_f16) ||
+        !aligned16(out))
+        return fail(QUAROT_ERR_MISALIGNED, "q, codes, scales and output must be 16-byte aligned");
+    int dev;
+    DeviceInfo *info;
+    quarot_status_t s = current_device(dev, info);
+    if (s != QUAROT_OK)
+        return s;
+    const __half *qh = static_cast<const __half *>(q_f16);
+    const __half *ksh = static_cast<const __half *>(ks_f16);
+    const __half *vsh = static_cast<const __half *>(vs_f16);
+    cudaStream_t st = (cudaStream_t)stream;
+    const int hkv = (int)Hkv;
+    switch (G) {
+    case 1: return launch_decode_tc<1>(qh, signs, kq, ksh, vq, vsh, B, T, hkv, out, st, dev);
+    case 2: return launch_decode_tc<2>(qh, signs, kq, ksh, vq, vsh, B, T, hkv, out, st, dev);
+    case 4: return launch_decode_tc<4>(qh, signs, kq, ksh, vq, vsh, B, T, hkv, out, st, dev);
+    case 8: return launch_decode_tc<8>(qh, signs, kq, ksh, vq, vsh, B, T, hkv, out, st, dev);
+    default: return launch_decode_tc<16>(qh, signs, kq, ksh, vq, vsh, B, T, hkv, out, st, dev);
+    }
 }
 
 quarot_status_t quarot_get_device_status(quarot_stream_t stream)

@@ -83,17 +83,6 @@ __device__ __forceinline__ bool pair_barrier_and(int id, bool p)
     return r != 0;
 }
 
-// Shared-memory descriptor of an MN-major operand in the 128-byte-swizzled
-// canonical layout: each K row holds 64 consecutive MN elements (128 bytes),
-// 8 K rows form a 1024-byte swizzle atom (stride byte offset 1024 between
-// groups of 8 K rows), and consecutive 64-element MN atoms lie `lbo` bytes
-// apart (leading byte offset).  Version 1, base offset 0, swizzle mode 2.
-__device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t saddr, uint32_t lbo)
-{
-    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(lbo >> 4) << 16) | ((uint64_t)(1024 >> 4) << 32) |
-           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-
 template <int LOGM, int GROUP, int BITS>
 __global__ void __launch_bounds__(kRtThreads, 1)
 had_tc_quant_kernel(const __grid_constant__ CUtensorMap tmap,   // x as fp16 [M * m, 128], box {64, 128}, SW128

@@ -174,3 +174,14 @@ def test_mma_probe_rejects(q):
     assert q.lib.quarot_probe_mma_i8(0, ctypes.byref(n), None) == 1
     assert q.lib.quarot_probe_mma_i8((1 << 22) + 1, ctypes.byref(n), None) == 1
     assert q.lib.quarot_probe_mma_i8(10, None, None) == 1
+
+
+def test_fused_decode_rejects(q):
+    f = q.lib.quarot_kv_decode_attention
+    assert f(A16, 64, A16, A16, A16, A16, A16, 1, 16, 8, 64, A16, None) == 2      # D != 128
+    assert f(A16, 12, A16, A16, A16, A16, A16, 1, 16, 8, 128, A16, None) == 2     # Hq % Hkv != 0
+    assert f(A16, 24, A16, A16, A16, A16, A16, 1, 16, 8, 128, A16, None) == 2     # group of 3
+    assert f(A16, 64, A16, A16, A16, A16, A16, 1, 0, 8, 128, A16, None) == 1      # no tokens
+    assert f(A16, 64, A16, A16, None, A16, A16, 1, 16, 8, 128, A16, None) == 1
+    assert f(A16, 64, A16, A16, A16, MIS, A16, 1, 16, 8, 128, A16, None) == 3
+    assert f(None, 64, None, None, None, None, None, 0, 16, 8, 128, None, None) == 0   # empty batch
