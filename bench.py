@@ -48,7 +48,8 @@ def parse():
     p.add_argument("--cpu-rows", type=int, default=2048, help="token rows of the CPU-baseline sample")
     p.add_argument("--case", choices=["gemm", "gemm_group", "gemm8", "gemm8_full", "gemm_asym", "rotate",
                                       "rotate_asym", "block", "kron", "kron_tok", "kvquant", "kvscores",
-                                      "kvattend", "kvattend_b64", "kvdecode", "kvdecode_b64", "i8peak"],
+                                      "kvattend", "kvattend_b64", "kvdecode", "kvdecode_b64", "i8peak",
+                                      "llama7b", "downproj"],
                    default=None, help="time one kernel on a capture-sized workload (for ncu), not the step")
     return p.parse_args()
 
@@ -213,6 +214,13 @@ def cpu_reference_step(w, c, rows, kv_batches, x, qw_codes, sw, s, kv):
     return full, desc, t_lin + t_kv
 
 
+def extrapolation(rows, M, kv_batches, B):
+    """How a timed CPU sample is scaled to the whole step: linearly in token
+    rows (linear layer) and in batches (KV cache)."""
+    return {"timed_token_rows": rows, "step_token_rows": M, "timed_kv_batches": kv_batches, "step_kv_batches": B,
+            "factor_linear": M / rows, "factor_kv": B / kv_batches}
+
+
 def cpu_inputs(w, c, kv_batches):
     import oracle
     from rotation_bit_quantization_randomized_b200 import synth
@@ -248,7 +256,9 @@ def run_reference(args, rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64/int64", "data": "synthetic",
         "config": {"workload": WORKLOAD},
-        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": cores, "kind": "oracle", "sample": desc},
+        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": cores, "kind": "oracle", "sample": desc,
+                         "extrapolated": extrapolation(rows, w.M, kvb, c.B)},
+        "extrapolated": extrapolation(rows, w.M, kvb, c.B),
         "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }))
 
@@ -407,7 +417,7 @@ def run_ours(args, rank, world, local_rank, dist):
         s2, qw_codes, sw2, kv = cpu_inputs(w, c, kvb)
         full_s, desc, spent = cpu_reference_step(w, c, rows, kvb, x_h, qw_codes, sw2, s2, kv)
         cpu = {"value": ops / full_s / 1e12, "unit": "TOPS", "cores": oracle.max_threads(), "kind": "oracle",
-               "sample": desc}
+               "sample": desc, "extrapolated": extrapolation(rows, w.M, kvb, c.B)}
 
     if rank == 0:
         line = {
@@ -446,6 +456,66 @@ def run_ours(args, rank, world, local_rank, dist):
         print(json.dumps(line))
 
 
+def run_linear_case(args, q, torch, dev):
+    """The 7B-shaped linears (2048 tokens, K 4096, H_4096 per token -> N 4096
+    and 11008) or the down-projection (2048 tokens, K 11008, I_86 x H_128 with
+    groups of 128 -> N 4096), on the seeded synthetic inputs of those
+    workloads.  These are L2-sized, so every timed iteration takes the next of
+    several buffer sets whose total exceeds twice the L2: no iteration finds
+    its inputs in L2.  Per kernel: CUDA events around each call."""
+    from rotation_bit_quantization_randomized_b200 import synth
+    w = synth.LLAMA2_7B if args.case == "llama7b" else synth.DOWN_PROJ
+    M, K = w.M, w.K
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    s = torch.from_numpy(synth.signs(K, w.seed)).to(dev)
+    x0 = torch.from_numpy(synth.activations(w)).to(dev)
+    Ws = {N: q.quarot_rotate_quant(torch.from_numpy(synth.weights(w, N)).to(dev), s, w.had_block, w.group)
+          for N in w.Ns}
+    set_bytes = x0.numel() * 2 + M * K // 2 + sum(N * K // 2 + M * N * 2 for N in w.Ns)
+    nsets = max(2, -(-3 * l2 // set_bytes))
+    sets = []
+    for _ in range(nsets):
+        qa = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+        sa = torch.empty((M,), dtype=torch.float32, device=dev) if w.group == 0 else \
+            torch.empty((M, K // 128), dtype=torch.float16, device=dev)
+        outs = {N: torch.empty((M, N), dtype=torch.float16, device=dev) for N in w.Ns}
+        wts = {N: (Ws[N][0].clone(), Ws[N][1].clone()) for N in w.Ns}
+        sets.append((x0.clone(), qa, sa, outs, wts))
+    stream = torch.cuda.current_stream()
+    n_ev = 1 + len(w.Ns)
+
+    def step(i, ev=None):
+        x, qa, sa, outs, wts = sets[i % nsets]
+        if ev is not None:
+            ev[0].record(stream)
+        q.quarot_rotate_quant(x, s, w.had_block, w.group, qa, sa)
+        if ev is not None:
+            ev[1].record(stream)
+        for j, N in enumerate(w.Ns):
+            q.quarot_int4_linear(qa, sa, wts[N][0], wts[N][1], w.group, outs[N])
+            if ev is not None:
+                ev[2 + j].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev + 1)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        step(i, evs[i])
+    torch.cuda.synchronize()
+    if q.quarot_get_device_status() != 0:
+        raise RuntimeError("device status not OK")
+    per = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(n_ev)] for e in evs]).mean(axis=0)
+    res = {"case": args.case, "workload": w.name, "buffer_sets": nsets,
+           "l2": f"{nsets} buffer sets of {set_bytes / 2**20:.0f} MiB in rotation (> 2 x L2 of {l2 / 2**20:.0f} MiB)",
+           "rotate_quant_ms": per[0], "rotate_quant_gbs": bytes_rotate_quant(M, K) / (per[0] * 1e-3) / 1e9,
+           "source_sha": source_hash()}
+    for j, N in enumerate(w.Ns):
+        res[f"int4_linear_N{N}_ms"] = per[1 + j]
+        res[f"int4_linear_N{N}_tops"] = 2.0 * M * N * K / (per[1 + j] * 1e-3) / 1e12
+    print(json.dumps(res))
+
+
 def run_case(args):
     """One kernel on a smaller, capture-sized case; random codes/values drawn on the device."""
     import torch
@@ -454,6 +524,9 @@ def run_case(args):
     dev = torch.device("cuda:0")
     g = torch.Generator(device=dev)
     g.manual_seed(1234)
+    if args.case in ("llama7b", "downproj"):
+        run_linear_case(args, q, torch, dev)
+        return
     if args.case in ("gemm", "gemm_group"):
         M, N, K = 4096, 28672, 8192
         group = 128 if args.case == "gemm_group" else 0
