@@ -148,11 +148,16 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
-def probe_i8_peak(q, torch, stream, launches=20, steps=20000):
+PROBE_OPERANDS = {0: "zero", 1: "random int8 bytes", 2: "random 4-bit codes in the high nibble"}
+
+
+def probe_i8_peak(q, torch, stream, launches=20, steps=20000, operands=0):
     """Dense tcgen05 kind::i8 rate (TOPS) of the probe kernel: MMAs of the GEMMs'
-    shape on operands resident in shared memory, timed with CUDA events on the
-    launching stream after one warm-up launch; with the median SM clock seen."""
-    q.quarot_probe_mma_i8(steps, stream)
+    shape on operands resident in shared memory (zeros, random bytes, or random
+    high-nibble 4-bit codes), timed with CUDA events on the launching stream
+    after one warm-up launch; with the median SM clock seen.  One launch of
+    20000 steps is ~5.4 ms at 1965 MHz."""
+    q.quarot_probe_mma_i8(steps, stream, operands)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -160,7 +165,7 @@ def probe_i8_peak(q, torch, stream, launches=20, steps=20000):
         e0.record(stream)
         ops = 0
         for _ in range(launches):
-            ops += q.quarot_probe_mma_i8(steps, stream)
+            ops += q.quarot_probe_mma_i8(steps, stream, operands)
         e1.record(stream)
         torch.cuda.synchronize()
     if q.quarot_get_device_status() != 0:
@@ -367,7 +372,13 @@ def run_ours(args, rank, world, local_rank, dist):
     ops = 2.0 * M * N * K
     value = job_rate(ops, world, ms_step * 1e-3) / 1e12
     pk = peaks()
-    i8_peak, i8_probe_ms, i8_clk = probe_i8_peak(q, torch, stream)
+    # the denominator: the probe on operands of the GEMM's own form (4-bit
+    # codes in the high nibble), run about as long as the timed region so that
+    # it meets the power limit as the step did; the zero-operand rate (no
+    # power limit reached) is kept beside it
+    i8_peak, i8_probe_ms, i8_clk = probe_i8_peak(q, torch, stream, operands=2,
+                                                 launches=max(20, int(np.ceil(total_ms / 5.4))))
+    i8_zero, _, i8_zero_clk = probe_i8_peak(q, torch, stream, operands=0)
     gemm_tops = ops / (k_ms[1] * 1e-3) / 1e12
     rq_gbs = bytes_rotate_quant(M, K) / (k_ms[0] * 1e-3) / 1e9
     kvq_gbs = bytes_kv_quant(c.B, c.T, c.Hkv, c.D) / (k_ms[2] * 1e-3) / 1e9
@@ -432,9 +443,15 @@ def run_ours(args, rank, world, local_rank, dist):
             "roofline": {"bound": "tensor", "kernel": "int4_gemm_pair_kernel<224,0> (quarot_int4_linear)",
                          "achieved": gemm_tops, "peak": i8_peak, "unit": "TFLOP/s",
                          "frac": gemm_tops / i8_peak, "traffic": traffic,
-                         "peak_note": ("dense int8 tensor rate measured in this run by the tcgen05 kind::i8 "
-                                       "probe (quarot_probe_mma_i8: M256 N256 K32 CTA-pair MMAs on resident "
-                                       f"operands, {i8_probe_ms:.0f} ms at median {i8_clk['sm_mhz']} MHz)"),
+                         "peak_note": ("of measured: dense int8 tensor rate measured in this run by the tcgen05 "
+                                       "kind::i8 probe (quarot_probe_mma_i8: M256 N256 K32 CTA-pair MMAs on "
+                                       "resident random 4-bit codes in the high nibble, the GEMM's operand form; "
+                                       f"{i8_probe_ms:.0f} ms, about the timed region's length, at median "
+                                       f"{i8_clk['sm_mhz']} MHz, reasons {i8_clk['reasons']})"),
+                         "peak_zero_operands": i8_zero,
+                         "frac_of_zero_operand_probe": gemm_tops / i8_zero,
+                         "zero_operand_note": ("the same probe on zero operands, 108 ms: no power limit "
+                                               f"reached, median {i8_zero_clk['sm_mhz']} MHz"),
                          "frac_of_nominal_4500": gemm_tops / 4500.0,
                          "frac_of_2x_bf16_burst": gemm_tops / (2.0 * pk["bf16"]),
                          "unit_note": "tera integer ops (2 per multiply-add), reported in the TFLOP/s field"},
@@ -542,9 +559,12 @@ def run_case(args):
         fn = lambda: q.quarot_int4_linear(qa, sa, qw, sw, group, out)
         work, unit = 2.0 * M * N * K / 1e12, "TOPS"
     elif args.case == "i8peak":
-        tops, ms, clk = probe_i8_peak(q, torch, torch.cuda.current_stream(), launches=args.steps)
-        print(json.dumps({"case": args.case, "ms": ms / args.steps, "TOPS": tops, "clocks": clk,
-                          "source_sha": source_hash()}))
+        res = {}
+        for operands, name in PROBE_OPERANDS.items():
+            tops, ms, clk = probe_i8_peak(q, torch, torch.cuda.current_stream(), launches=args.steps,
+                                          operands=operands)
+            res[name] = {"ms_per_launch": ms / args.steps, "TOPS": tops, "clocks": clk}
+        print(json.dumps({"case": args.case, "launches": args.steps, "probe": res, "source_sha": source_hash()}))
         return
     elif args.case in ("gemm8", "gemm8_full"):
         M, N, K = (4096 if args.case == "gemm8" else 32768), 28672, 8192

@@ -484,9 +484,16 @@ quarot_status_t quarot_get_device_status(quarot_stream_t stream);
  * waits for them; nothing is copied or stored.  *pairs receives the number of
  * CTA pairs launched, so one call performs pairs * steps * 4 * 2 * 256 * 256
  * * 32 integer operations; timing the call on `stream` gives the dense INT8
- * tensor rate.  Limits: 1 <= steps <= 2^22.
+ * tensor rate.  operands: 0 fills both operands with zeros, 1 with
+ * pseudo-random bytes (the INT8 GEMMs' codes), 2 with pseudo-random 4-bit
+ * codes in the high nibble of each byte (the form in which the INT4 GEMMs
+ * hand their codes to the tensor core).  The work per clock is the same for
+ * all three; nonzero operands draw the power that real data draws, so that a
+ * run of them shows the rate the board's power limit allows.  Limits:
+ * 1 <= steps <= 2^22; operands in {0, 1, 2}.
  */
-quarot_status_t quarot_probe_mma_i8(int64_t steps, int64_t *pairs, quarot_stream_t stream);
+quarot_status_t quarot_probe_mma_i8(int64_t steps, int operands, int64_t *pairs,
+                                    quarot_stream_t stream);
 
 /*
  * quarot_test_wait_timeout -- exercises the bounded-wait path of the kernels

@@ -51,7 +51,7 @@ _SIGS = {
     "quarot_kron_factor": ([_I64, _P], _INT),
     "quarot_kv_decode_attend": ([_P, _I64, _I64, _P, _P, _I64, _I64, _I64, _P, _P], _INT),
     "quarot_kv_decode_attention": ([_P, _I64, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P], _INT),
-    "quarot_probe_mma_i8": ([_I64, _P, _P], _INT),
+    "quarot_probe_mma_i8": ([_I64, _INT, _P, _P], _INT),
     "quarot_test_wait_timeout": ([_P, _I64, _P, _P, _I64, ctypes.c_uint64, _P], _INT),
     "quarot_get_device_status": ([_P], _INT),
     "quarot_status_string": ([_INT], ctypes.c_char_p),
@@ -393,11 +393,12 @@ def quarot_kv_decode_attention(q: torch.Tensor, signs: torch.Tensor, kq: torch.T
     return out
 
 
-def quarot_probe_mma_i8(steps: int, stream=None) -> int:
-    """Launches the dense INT8 tensor-pipe probe; returns the integer
-    operations it performs (time it on the stream with CUDA events)."""
+def quarot_probe_mma_i8(steps: int, stream=None, operands: int = 0) -> int:
+    """Launches the dense INT8 tensor-pipe probe on zero (0), pseudo-random
+    byte (1) or pseudo-random high-nibble 4-bit (2) operands; returns the
+    integer operations it performs (time it on the stream with CUDA events)."""
     pairs = ctypes.c_int64(0)
-    _check("quarot_probe_mma_i8", lib.quarot_probe_mma_i8(steps, ctypes.byref(pairs), _stream(stream)))
+    _check("quarot_probe_mma_i8", lib.quarot_probe_mma_i8(steps, operands, ctypes.byref(pairs), _stream(stream)))
     return int(pairs.value) * steps * 4 * 2 * 256 * 256 * 32
 
 

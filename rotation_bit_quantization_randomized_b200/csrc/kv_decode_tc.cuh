@@ -23,8 +23,8 @@
 // where row n < G of B is head n's hi part and row G + n its lo part (rows
 // past 2 G, when G < 8, only feed accumulator columns that are never read).  A_k
 // (key codes, K-major) and A_v (value codes, MN-major: the dims of a token
-// are contiguous) share one 128 x 128 fp16 tile layout in shared memory, so
-// one conversion routine serves both; it emits the dims of every group of
+// are contiguous) have the same 128 x 128 fp16 tile layout in shared memory
+// (two tiles), so one conversion routine serves both; it emits the dims of every group of
 // four in the order (0, 2, 1, 3) (two nibble bytes become a low-nibble and a
 // high-nibble half2 word), and the query rows use the same order, so each dot
 // product is unchanged and output lane p holds dim d(p).
@@ -32,18 +32,19 @@
 // A cluster of S CTAs covers one (batch, KV head); CTA r walks its slice of
 // the tokens in tiles of 128 with the running-maximum softmax (in base 2: the
 // scores carry the factor log2(e) / sqrt(128) and the exponentials are exp2):
-// per tile the key codes are converted and multiplied, the 128 threads (one
-// per token) read their scores, the tile maximum updates the running maximum
-// m and the sum l, the value accumulator D_o is rescaled in tensor memory when
-// m grows, the weights e * vs (one power-of-two scale for the whole slice,
-// from its largest value scale) are written as B_w, and the value codes
-// (converted into the same tile) are multiplied into D_o.  The next
-// tile's codes arrive by asynchronous copies meanwhile.  At the end the CTAs
-// of the cluster combine their (m, l, acc) through distributed shared memory:
-// out = sum_r exp(m_r - M) acc_r / sum_r exp(m_r - M) l_r, M = max_r m_r.
-// Several CTAs share an SM (about 60 KB of shared memory and 32 or 64
-// tensor-memory columns each), so one CTA's conversions overlap another's
-// waits.  Every wait is bounded.
+// per tile the key codes are converted and multiplied, the value codes are
+// converted while those MMAs run, the 128 threads (one per token) read their
+// scores, the tile maximum updates the running maximum m and the sum l, the
+// value accumulator D_o is rescaled in tensor memory when m grows, the
+// weights e * vs (one power-of-two scale for the whole slice, from its
+// largest value scale) are written as B_w, and the value MMAs into D_o run
+// while the next tile's keys are converted.  Each thread loads its token's
+// key and value rows of the next tile into registers one tile ahead.  At the
+// end the CTAs of the cluster combine their (m, l, acc) through distributed
+// shared memory: out = sum_r exp(m_r - M) acc_r / sum_r exp(m_r - M) l_r,
+// M = max_r m_r.  Several CTAs share an SM (about 73 KB of shared memory and
+// 32 or 64 tensor-memory columns each), so one CTA's conversions overlap
+// another's waits.  Every wait is bounded.
 #pragma once
 
 #include "common.cuh"
@@ -62,13 +63,13 @@ template <int G>
 struct DecShape {
     static constexpr int NP = G <= 8 ? 16 : 32;            // MMA N: G hi rows, G lo rows, zero padding
     static constexpr int kTmemCols = G <= 8 ? 32 : 64;     // D_s at column 0, D_o at column NP
-    static constexpr int kTileOff = 0;                     // code tile: 2 panels of 128 rows x 128 B
-    static constexpr int kBqOff = 32768;                   // B_q: 2 panels of NP rows x 128 B
+    static constexpr int kKTileOff = 0;                    // key tile: 2 panels of 128 rows x 128 B
+    static constexpr int kVTileOff = 32768;                // value tile, the same shape
+    static constexpr int kBqOff = 65536;                   // B_q: 2 panels of NP rows x 128 B
     static constexpr int kBwOff = kBqOff + 2 * NP * 128;   // B_w: the same shape
-    static constexpr int kStageBytes = 2 * kDecTile * 64;  // raw codes of one tile: K then V, 64 B a token
-    static constexpr int kStageOff = kBwOff + 2 * NP * 128; // two stages: tiles j + 1 and j + 2 in flight
-    static constexpr int kMiscOff = kStageOff + 2 * kStageBytes;
-    // misc: mbarrier (8), tmem slot (4), pad (4), drain mbarrier (8), pad, then floats:
+    static constexpr int kMiscOff = kBwOff + 2 * NP * 128;
+    // misc: key mbarrier (8), tmem slot (4), pad (4), drain mbarrier (8),
+    // value mbarrier (8), then floats:
     //   red[4][G + 1]  per-warp tile maxima of each head's scores
     //   m[G], l[G], lpart[4][G], inv_qs[G], vmx[4]
     static constexpr int kRedOff = kMiscOff + 32;
@@ -79,10 +80,11 @@ struct DecShape {
     static constexpr int kIqOff = kLpOff + 4 * G * 4;       // 1 / 2^e of each head's query
     static constexpr int kVmOff = kIqOff + G * 4;           // per-warp maxima of the slice's value scales
     static constexpr int kBytes = kVmOff + 16 + 1024;
-    // the code tile is free after the last tile: the CTA's unnormalized
+    // the key tile is free after the last tile: the CTA's unnormalized
     // result fin[G][128] fp32 lives there then
-    static constexpr int kFinOff = kTileOff;
-    static_assert(kBqOff % 1024 == 0 && kBwOff % 1024 == 0 && kStageOff % 16 == 0, "alignment");
+    static constexpr int kFinOff = kKTileOff;
+    static_assert(kBqOff % 1024 == 0 && kBwOff % 1024 == 0 && kMiscOff % 16 == 0, "alignment");
+    static_assert(G * 128 * 4 <= 32768, "fin fits the key tile");
 };
 
 // dim held by position p of a converted row: (0, 2, 1, 3) within each group of four
@@ -139,6 +141,43 @@ __device__ __forceinline__ void dec_put_split(uint8_t *b, int n, int k, float xs
     *at(G + n) = lo;
 }
 
+// The maxima over a warp's 32 tokens of each of the G heads' scores, into
+// red_w[g].  Halving exchanges: at the level of lane bit m the two partners
+// keep complementary halves of the values still held, each taking the larger
+// of its own and the partner's value for the half it keeps; after log2(G)
+// levels every lane holds one head's partial maximum, and plain butterfly
+// levels over the remaining lane bits finish it (G - 1 + 5 - log2(G)
+// shuffles instead of 5 G).
+template <int G>
+__device__ __forceinline__ void dec_tile_max(const float (&s)[G], float *red_w, int lane)
+{
+    constexpr int L = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : G == 8 ? 3 : 4;
+    static_assert((1 << L) == G, "G is a power of two up to 16");
+    float v[G];
+#pragma unroll
+    for (int i = 0; i < G; ++i)
+        v[i] = s[i];
+    int g = 0;
+#pragma unroll
+    for (int lv = 0; lv < L; ++lv) {
+        const int mask = 16 >> lv;
+        const int half = G >> (lv + 1);
+        const bool upper = (lane & mask) != 0;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+            const float send = upper ? v[i] : v[half + i];
+            const float keep = upper ? v[half + i] : v[i];
+            v[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, mask));
+        }
+        g += upper ? half : 0;
+    }
+#pragma unroll
+    for (int mask = 16 >> L; mask >= 1; mask >>= 1)
+        v[0] = fmaxf(v[0], __shfl_xor_sync(0xffffffffu, v[0], mask));
+    if ((lane & ((32 >> L) - 1)) == 0)
+        red_w[g] = v[0];
+}
+
 // Power of two 2^e that brings max|x| (> 0) into [2^14, 2^15): hi parts then
 // stay far from fp16 overflow and lo parts keep 11 more bits.  Built from the
 // exponent bits, so 2^e and its inverse are exact; 1 for a zero maximum.
@@ -155,7 +194,7 @@ __device__ __forceinline__ float dec_pow2_scale(float amax, float &inv)
 }
 
 template <int G>
-__global__ void __launch_bounds__(kDecThreads)
+__global__ void __launch_bounds__(kDecThreads, G <= 8 ? 3 : 2)
 kv_decode_tc_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
                     const int8_t *__restrict__ signs,    // [Hkv, 128]
                     const uint8_t *__restrict__ kq,      // [B, T, Hkv, 64 bytes]
@@ -168,13 +207,14 @@ kv_decode_tc_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
     constexpr int NP = S::NP;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *tile = smem + S::kTileOff;
+    uint8_t *ktile = smem + S::kKTileOff;
+    uint8_t *vtile = smem + S::kVTileOff;
     uint8_t *bq = smem + S::kBqOff;
     uint8_t *bw = smem + S::kBwOff;
-    uint8_t *stages = smem + S::kStageOff;
-    const uint32_t bar = smem_u32(smem + S::kMiscOff);
+    const uint32_t bar_s = smem_u32(smem + S::kMiscOff);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + S::kMiscOff + 8);
     const uint32_t bar_drain = smem_u32(smem + S::kMiscOff + 16);
+    const uint32_t bar_o = smem_u32(smem + S::kMiscOff + 24);
     float *red = reinterpret_cast<float *>(smem + S::kRedOff);      // [4][G + 1]
     float *sm_m = reinterpret_cast<float *>(smem + S::kMOff);
     float *sm_l = reinterpret_cast<float *>(smem + S::kLOff);
@@ -198,7 +238,8 @@ kv_decode_tc_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
     const int ntiles = (int)((te - ts + kDecTile - 1) / kDecTile);
 
     if (tid == 0) {
-        mbar_init(bar, 1);
+        mbar_init(bar_s, 1);
+        mbar_init(bar_o, 1);
         mbar_init(bar_drain, 1);
         mbar_fence_init();
     }
@@ -206,31 +247,30 @@ kv_decode_tc_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
         tmem_alloc(smem_u32(tmem_slot), S::kTmemCols);
         tmem_relinquish();
     }
-    // raw codes of tile j into stage j % 2: thread t copies token t's key and
-    // value rows; every call commits one group (empty past the last tile), so
-    // that "all but the latest group done" always means "tile j has landed"
-    auto issue_copy = [&](int j) {
+    // thread t holds token t's key and value rows of the next tile in
+    // registers: loaded one tile ahead, converted into the tiles when due
+    auto load_row = [&](const uint8_t *src, int j, uint4 (&w)[4]) {
         const int64_t t = ts + (int64_t)j * kDecTile + tid;
-        uint8_t *stage = stages + (j & 1) * S::kStageBytes;
-        const uint32_t dk = smem_u32(stage + tid * 64), dv = smem_u32(stage + kDecTile * 64 + tid * 64);
         if (j < ntiles && t < te) {
-            const uint8_t *sk = kq + ((b * T + t) * Hkv + h) * 64;
-            const uint8_t *sv = vq + ((b * T + t) * Hkv + h) * 64;
+            const uint4 *p = reinterpret_cast<const uint4 *>(src + ((b * T + t) * Hkv + h) * 64);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                cp_async16(dk + 16 * c, sk + 16 * c);
-                cp_async16(dv + 16 * c, sv + 16 * c);
-            }
+            for (int c = 0; c < 4; ++c)
+                w[c] = __ldg(p + c);
+        } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                w[c] = make_uint4(0u, 0u, 0u, 0u);
         }
-        asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    issue_copy(0);
-    issue_copy(1);
+    uint4 krow[4], vrow[4];
+    load_row(kq, 0, krow);
+    load_row(vq, 0, vrow);
 
     // ---- the slice's largest value scale (the weights e * vs never exceed
     // it, so one power-of-two scale serves every tile of the slice)
     {
         float vm = 0.f;
+#pragma unroll 4
         for (int j = 0; j < ntiles; ++j) {
             const int64_t t = ts + (int64_t)j * kDecTile + tid;
             if (t < te)
@@ -323,12 +363,12 @@ kv_decode_tc_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
         lsum[g] = 0.f;
         m_run[g] = -INFINITY;
     }
-    uint32_t commits = 0;
+    uint32_t commits_s = 0, commits_o = 0;
     bool ok = true;
     constexpr uint32_t idesc_s = idesc_f16(128, NP);
     constexpr uint32_t idesc_o = idesc_f16(128, NP) | (1u << 15);    // A (values) MN-major
-    auto mma_wait = [&]() {
-        // the latest commit has completed (bounded; the CTA then gives up as a whole)
+    auto mma_wait = [&](uint32_t bar, uint32_t commits) {
+        // the latest commit to `bar` has completed (bounded; the CTA then gives up as a whole)
         bool done = true;
         if (!mbar_try_wait(bar, (commits - 1) & 1)) {
             const uint64_t t0 = globaltimer_ns();
@@ -352,40 +392,39 @@ kv_decode_tc_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
     };
     float ks_next, vs_next;
     load_scales(0, ks_next, vs_next);
+    // Per tile j: keys converted -> score MMAs issued -> (value MMAs of tile
+    // j - 1 done) values converted while the score MMAs run -> scores, softmax
+    // weights -> value MMAs issued, running while the next tile's keys are
+    // converted.  The key tile is free at the top of an iteration (its MMAs
+    // were waited for before the scores were read).
 #pragma unroll 1
     for (int j = 0; j < ntiles && ok; ++j) {
         const int64_t t = ts + (int64_t)j * kDecTile + tid;
         const bool tv = t < te;
         const float ksv = ks_next, vsv = vs_next;
         load_scales(j + 1, ks_next, vs_next);
-        const uint8_t *stage = stages + (j & 1) * S::kStageBytes;
-        // the previous tile's value MMAs are done with the code tile
-        if (j > 0 && !(ok = mma_wait()))
-            break;
-        asm volatile("cp.async.wait_group 1;" ::: "memory");
-        __syncthreads();
         // ---- keys: convert, multiply with the query rows
-        {
-            uint4 w[4];
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                w[c] = tv ? *reinterpret_cast<const uint4 *>(stage + tid * 64 + 16 * c)
-                          : make_uint4(0u, 0u, 0u, 0u);
-            dec_convert_row(w, tile, tid);
-        }
+        dec_convert_row(krow, ktile, tid);
+        load_row(kq, j + 1, krow);
         fence_proxy_async_smem();
         __syncthreads();
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-                umma_f16_ss(tmem, desc_kmajor_sw128(smem_u32(tile) + 16384 * (kk >> 2) + 32 * (kk & 3)),
+                umma_f16_ss(tmem, desc_kmajor_sw128(smem_u32(ktile) + 16384 * (kk >> 2) + 32 * (kk & 3)),
                             desc_kmajor_sw128(smem_u32(bq) + NP * 128 * (kk >> 2) + 32 * (kk & 3)), idesc_s,
                             kk > 0 ? 1u : 0u);
-            umma_commit(bar);
+            umma_commit(bar_s);
         }
-        ++commits;
-        if (!(ok = mma_wait()))
+        ++commits_s;
+        // ---- values: the previous tile's value MMAs are done with the value
+        // tile and B_w; convert while the score MMAs run
+        if (j > 0 && !(ok = mma_wait(bar_o, commits_o)))
+            break;
+        dec_convert_row(vrow, vtile, tid);
+        load_row(vq, j + 1, vrow);
+        if (!(ok = mma_wait(bar_s, commits_s)))
             break;
         tc_fence_after();
         // ---- scores of token t (lane t of D_s), the tile maxima
@@ -409,12 +448,7 @@ kv_decode_tc_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
                 s[g] = tv ? x * km : -INFINITY;
             }
         }
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const float mg = warp_max(s[g], 32);
-            if (lane == 0)
-                red[warp * (G + 1) + g] = mg;
-        }
+        dec_tile_max<G>(s, red + warp * (G + 1), lane);
         __syncthreads();
         float beta[G];                               // rescale of the value accumulator
         bool rescale = false;
@@ -453,34 +487,22 @@ kv_decode_tc_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
                 tmem_st32(lane_base + NP, *reinterpret_cast<uint32_t (*)[32]>(d));
             tmem_wait_st();
         }
-        // ---- values: convert into the same tile (the key MMAs are done)
-        {
-            uint4 w[4];
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                w[c] = tv ? *reinterpret_cast<const uint4 *>(stage + kDecTile * 64 + tid * 64 + 16 * c)
-                          : make_uint4(0u, 0u, 0u, 0u);
-            dec_convert_row(w, tile, tid);
-        }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
-        // stage j % 2 is consumed: tile j + 2 may land there
-        issue_copy(j + 2);
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-                umma_f16_ss(tmem + NP, desc_mnmajor_sw128(smem_u32(tile) + 2048 * kk, 16384),
+                umma_f16_ss(tmem + NP, desc_mnmajor_sw128(smem_u32(vtile) + 2048 * kk, 16384),
                             desc_kmajor_sw128(smem_u32(bw) + NP * 128 * (kk >> 2) + 32 * (kk & 3)), idesc_o,
                             (j > 0 || kk > 0) ? 1u : 0u);
-            umma_commit(bar);
+            umma_commit(bar_o);
         }
-        ++commits;
+        ++commits_o;
     }
     if (ok && ntiles > 0)
-        ok = mma_wait();
-    asm volatile("cp.async.wait_all;" ::: "memory");
+        ok = mma_wait(bar_o, commits_o);
 
     // ---- this CTA's partial result: fin[g][d] (unnormalized), m, l
     if (ok && ntiles > 0) {

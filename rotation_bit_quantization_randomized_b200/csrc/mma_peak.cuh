@@ -6,6 +6,13 @@
 // every CTA pair issues `steps` groups of four MMAs (one 128-byte K block)
 // into one accumulator and waits for them at the end; the results are never
 // read.  One CTA per SM (the shared-memory request keeps a second one off).
+//
+// The operands are all zero, pseudo-random bytes, or pseudo-random 4-bit
+// codes held in the high nibble of each byte (the form in which the INT4
+// GEMMs hand their codes to the tensor core).  The work per clock is the same
+// for all three, but the power drawn is not: nonzero operands toggle the
+// multipliers as real data does, and under the board's power limit the SM
+// clock, and with it the rate per second, settles lower than with zeros.
 #pragma once
 
 #include "int4_gemm.cuh"
@@ -23,8 +30,20 @@ struct MmaPeakShape {
     static_assert(kMiscOffset + 16 + 1024 <= kSmemBytes, "layout fits");
 };
 
+// MurmurHash3's 32-bit finalizer (Appleby): a bijective mix of a counter
+// into well-spread bits, here only a source of operand bytes.
+__device__ __forceinline__ uint32_t fmix32(uint32_t h)
+{
+    h ^= h >> 16;
+    h *= 0x85ebca6bu;
+    h ^= h >> 13;
+    h *= 0xc2b2ae35u;
+    h ^= h >> 16;
+    return h;
+}
+
 __global__ void __launch_bounds__(MmaPeakShape::kThreads, 1)
-mma_peak_i8_kernel(int64_t steps)
+mma_peak_i8_kernel(int64_t steps, int operands)
 {
     using S = MmaPeakShape;
     extern __shared__ uint8_t smem_raw[];
@@ -35,9 +54,19 @@ mma_peak_i8_kernel(int64_t steps)
     const int warp = threadIdx.x >> 5;
     const bool leader = cluster_ctarank() == 0;
 
-    // operands: any bytes will do; zeros keep the accumulator exact
-    for (int i = threadIdx.x; i < 2 * S::kTile / 16; i += S::kThreads)
-        reinterpret_cast<uint4 *>(smem)[i] = make_uint4(0u, 0u, 0u, 0u);
+    // operands: zeros, or bytes mixed from (CTA, word index), optionally with
+    // the low nibbles cleared; the int32 accumulation of random products
+    // wraps, which nothing reads
+    const uint32_t keep = operands == 2 ? 0xf0f0f0f0u : 0xffffffffu;
+    for (int i = threadIdx.x; i < 2 * S::kTile / 16; i += S::kThreads) {
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (operands != 0) {
+            const uint32_t c = (blockIdx.x * (2u * S::kTile / 16u) + (uint32_t)i) * 4u;
+            v = make_uint4(fmix32(c + 1u) & keep, fmix32(c + 2u) & keep, fmix32(c + 3u) & keep,
+                           fmix32(c + 4u) & keep);
+        }
+        reinterpret_cast<uint4 *>(smem)[i] = v;
+    }
     fence_proxy_async_smem();
     if (threadIdx.x == 0) {
         mbar_init(bar_done, 1);

@@ -808,42 +808,61 @@ quarot_status_t attend_resident_clusters(int G, int split, int dev, int &fit)
 }
 
 // Clusters of `split` fused decode CTAs (G query heads per KV head) that can
-// be resident at once, queried once per (device, G, split); also raises the
-// kernel's dynamic shared-memory limit.
+// be resident at once, computed once per (device, G); also raises the
+// kernel's dynamic shared-memory limit.  The count comes from the kernel's
+// own resources (shared memory with the per-CTA reservation, registers in
+// 256-register warp allocations, threads, CTA slots): the runtime's occupancy
+// queries report one CTA per SM for this kernel at any shared-memory size,
+// while up to three are resident when it runs (counted on B200 with %smid).
 template <int G>
 quarot_status_t decode_resident_clusters(int split, int dev, int &fit)
 {
-    static int cache[kMaxDevices][4];
-    static bool known[kMaxDevices][4];
-    const int si = split == 1 ? 0 : split == 2 ? 1 : split == 4 ? 2 : 3;
+    static int cache[kMaxDevices];
+    static bool known[kMaxDevices];
+    int per_sm = 0, sms = 0;
     {
         std::lock_guard<std::mutex> lk(g_mutex);
-        if (known[dev][si]) {
-            fit = cache[dev][si];
-            return QUAROT_OK;
-        }
+        if (known[dev])
+            per_sm = cache[dev];
     }
-    cudaError_t e = cudaFuncSetAttribute(kv_decode_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)DecShape<G>::kBytes);
+    cudaError_t e;
+    if (per_sm == 0) {
+        e = cudaFuncSetAttribute(kv_decode_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)DecShape<G>::kBytes);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cudaFuncSetAttribute");
+        // all of the unified L1 / shared storage as shared memory, so that
+        // several CTAs (about 75 KB each) share an SM
+        e = cudaFuncSetAttribute(kv_decode_tc_kernel<G>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cudaFuncSetAttribute");
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, kv_decode_tc_kernel<G>);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cudaFuncGetAttributes");
+        int smem_sm = 0, smem_res = 0, regs_sm = 0, thr_sm = 0, blk_sm = 0;
+        if (cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&smem_res, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&thr_sm, cudaDevAttrMaxThreadsPerMultiProcessor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&blk_sm, cudaDevAttrMaxBlocksPerMultiprocessor, dev) != cudaSuccess)
+            return fail(QUAROT_ERR_CUDA, "cudaDeviceGetAttribute failed");
+        const int warp_regs = ((fa.numRegs * 32 + 255) / 256) * 256;
+        const int cta_regs = warp_regs * (kDecThreads / 32);
+        const int cta_smem = (int)DecShape<G>::kBytes + (int)fa.sharedSizeBytes + smem_res;
+        per_sm = std::min(std::min(smem_sm / cta_smem, regs_sm / std::max(cta_regs, 1)),
+                          std::min(thr_sm / kDecThreads, blk_sm));
+        if (per_sm < 1)
+            return fail(QUAROT_ERR_CUDA, "kv_decode_tc_kernel does not fit on an SM");
+        std::lock_guard<std::mutex> lk(g_mutex);
+        cache[dev] = per_sm;
+        known[dev] = true;
+    }
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess)
-        return cuda_fail(e, "cudaFuncSetAttribute");
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)split, 1, 1);
-    cfg.blockDim = dim3(kDecThreads);
-    cfg.dynamicSmemBytes = DecShape<G>::kBytes;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)split;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaOccupancyMaxActiveClusters(&fit, kv_decode_tc_kernel<G>, &cfg);
-    if (e != cudaSuccess)
-        return cuda_fail(e, "cudaOccupancyMaxActiveClusters");
-    std::lock_guard<std::mutex> lk(g_mutex);
-    cache[dev][si] = fit;
-    known[dev][si] = true;
+        return cuda_fail(e, "cudaDeviceGetAttribute");
+    fit = sms * per_sm / split;
     return QUAROT_OK;
 }
 
@@ -852,24 +871,27 @@ quarot_status_t launch_decode_tc(const __half *q, const int8_t *signs, const uin
                                  const uint8_t *vq, const __half *vs, int64_t B, int64_t T, int Hkv, float *out,
                                  cudaStream_t st, int dev)
 {
-    // tokens split over a cluster of S CTAs, at least 128 tokens each: the S
-    // whose B * Hkv * S CTAs fill the resident slots best, then the one with
-    // fewer waves
+    // tokens split over a cluster of S CTAs, at least 128 tokens each.  A
+    // CTA's time is about its tiles plus a fixed part (query rotation, the
+    // cluster combine) that grows with S: 0.65 (1 + log2 S) tiles, as timed on
+    // B200 at T 2048 for B 1 .. 64; the launch takes about ceil(clusters /
+    // resident clusters) such CTA times.  The S with the smallest estimate.
     const int smax = T >= 1024 ? 8 : T >= 512 ? 4 : T >= 256 ? 2 : 1;
     int split = smax;
-    double best_eff = -1.0;
-    int64_t best_waves = 0;
-    for (int sp = smax; sp >= 1; sp /= 2) {
+    double best = 0.0;
+    for (int sp = 1, lg = 0; sp <= smax; sp *= 2, ++lg) {
         int fit = 0;
         quarot_status_t s = decode_resident_clusters<G>(sp, dev, fit);
         if (s != QUAROT_OK)
             return s;
+        if (fit <= 0)
+            continue;
         const int64_t clusters = B * Hkv;
-        const int64_t waves = fit > 0 ? (clusters + fit - 1) / fit : clusters;
-        const double eff = fit > 0 ? (double)clusters / ((double)waves * fit) : 0.0;
-        if (eff > best_eff + 1e-9 || (eff > best_eff - 1e-9 && waves < best_waves)) {
-            best_eff = eff;
-            best_waves = waves;
+        const int64_t waves = (clusters + fit - 1) / fit;
+        const int64_t tiles = ((T + sp - 1) / sp + kDecTile - 1) / kDecTile;
+        const double est = (double)waves * ((double)tiles + 0.65 * (1 + lg));
+        if (sp == 1 || est < best) {
+            best = est;
             split = sp;
         }
     }
@@ -1402,10 +1424,12 @@ quarot_status_t quarot_kv_decode_attend(const float *scores, int64_t B, int64_t 
     return after_launch("kv_attend_kernel launch");
 }
 
-quarot_status_t quarot_probe_mma_i8(int64_t steps, int64_t *pairs, quarot_stream_t stream)
+quarot_status_t quarot_probe_mma_i8(int64_t steps, int operands, int64_t *pairs, quarot_stream_t stream)
 {
     if (steps < 1 || steps > (int64_t(1) << 22))
         return fail(QUAROT_ERR_INVALID_ARG, "steps must lie in [1, 2^22]");
+    if (operands < 0 || operands > 2)
+        return fail(QUAROT_ERR_INVALID_ARG, "operands must be 0 (zeros), 1 (random bytes) or 2 (random 4-bit codes)");
     if (!pairs)
         return fail(QUAROT_ERR_INVALID_ARG, "null pointer");
     int dev;
@@ -1431,7 +1455,7 @@ quarot_status_t quarot_probe_mma_i8(int64_t steps, int64_t *pairs, quarot_stream
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, mma_peak_i8_kernel, steps);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, mma_peak_i8_kernel, steps, operands);
     if (e != cudaSuccess)
         return cuda_fail(e, "mma_peak_i8_kernel launch");
     *pairs = clusters;

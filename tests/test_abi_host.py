@@ -171,9 +171,12 @@ def test_timeout_entry_rejects(q):
 
 def test_mma_probe_rejects(q):
     n = ctypes.c_int64(0)
-    assert q.lib.quarot_probe_mma_i8(0, ctypes.byref(n), None) == 1
-    assert q.lib.quarot_probe_mma_i8((1 << 22) + 1, ctypes.byref(n), None) == 1
-    assert q.lib.quarot_probe_mma_i8(10, None, None) == 1
+    assert q.lib.quarot_probe_mma_i8(0, 0, ctypes.byref(n), None) == 1
+    assert q.lib.quarot_probe_mma_i8((1 << 22) + 1, 1, ctypes.byref(n), None) == 1
+    assert q.lib.quarot_probe_mma_i8(10, 0, None, None) == 1
+    assert q.lib.quarot_probe_mma_i8(10, 3, ctypes.byref(n), None) == 1
+    assert q.lib.quarot_probe_mma_i8(10, -1, ctypes.byref(n), None) == 1
+    assert "operands" in q.lib.quarot_last_error().decode()
 
 
 def test_fused_decode_rejects(q):
