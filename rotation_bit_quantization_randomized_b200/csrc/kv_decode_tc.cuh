@@ -54,7 +54,8 @@
 
 namespace quarot {
 
-constexpr int kDecThreads = 128;
+constexpr int kDecCompute = 128;                 // warps 0-3: one thread per token of a tile
+constexpr int kDecThreads = kDecCompute + 32;    // warp 4 issues the MMAs
 constexpr int kDecTile = 128;                    // tokens per tile
 constexpr int kDecMaxSplit = 8;
 constexpr uint64_t kDecWaitLimitNs = 2000000000ull;
@@ -68,11 +69,12 @@ struct DecShape {
     static constexpr int kBqOff = 65536;                   // B_q: 2 panels of NP rows x 128 B
     static constexpr int kBwOff = kBqOff + 2 * NP * 128;   // B_w: the same shape
     static constexpr int kMiscOff = kBwOff + 2 * NP * 128;
-    // misc: key mbarrier (8), tmem slot (4), pad (4), drain mbarrier (8),
-    // value mbarrier (8), then floats:
+    // misc: mbarriers "scores done" (8), tmem slot (4), pad (4), drain (8),
+    // "values done" (8), "key tile ready" (8), "value tile ready" (8), abort
+    // flag (4), pad, then floats:
     //   red[4][G + 1]  per-warp tile maxima of each head's scores
     //   m[G], l[G], lpart[4][G], inv_qs[G], vmx[4]
-    static constexpr int kRedOff = kMiscOff + 32;
+    static constexpr int kRedOff = kMiscOff + 64;
     static constexpr int kQmaxOff = kRedOff + 4 * (G + 1) * 4;
     static constexpr int kMOff = kQmaxOff + 4 * G * 4;
     static constexpr int kLOff = kMOff + G * 4;
@@ -80,11 +82,13 @@ struct DecShape {
     static constexpr int kIqOff = kLpOff + 4 * G * 4;       // 1 / 2^e of each head's query
     static constexpr int kVmOff = kIqOff + G * 4;           // per-warp maxima of the slice's value scales
     static constexpr int kBytes = kVmOff + 16 + 1024;
-    // the key tile is free after the last tile: the CTA's unnormalized
-    // result fin[G][128] fp32 lives there then
-    static constexpr int kFinOff = kKTileOff;
+    // the value tile is free after the last tile: there every CTA of the
+    // cluster receives, for the heads it finishes, the other CTAs' partial
+    // results: recv[rank][slot][128] fp32, then their m and l
+    static constexpr int kOwnMax = G;                          // heads one CTA finishes, at most
+    static constexpr int kRecvOff = kVTileOff;
+    static constexpr int kRecvMlOff = kVTileOff + 16384;
     static_assert(kBqOff % 1024 == 0 && kBwOff % 1024 == 0 && kMiscOff % 16 == 0, "alignment");
-    static_assert(G * 128 * 4 <= 32768, "fin fits the key tile");
 };
 
 // dim held by position p of a converted row: (0, 2, 1, 3) within each group of four
@@ -178,6 +182,61 @@ __device__ __forceinline__ void dec_tile_max(const float (&s)[G], float *red_w, 
         red_w[g] = v[0];
 }
 
+// 2^x by the SM's base-2 exponential instruction (ex2.approx, subnormal
+// results flushed to zero): the softmax weights and their rescale factors.
+// Its relative error is a few units in the last place of fp32; a weight's
+// error moves the normalized output by at most twice that relative error
+// times the largest value, and a rescale factor's error cancels, because the
+// accumulator and the sum of weights are scaled by the same computed factor.
+__device__ __forceinline__ float dec_exp2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Barrier of the four compute warps (named barrier 1, 128 threads); the MMA
+// warp never takes part.
+__device__ __forceinline__ void dec_bar_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// The same barrier, returning the AND of every compute thread's predicate.
+__device__ __forceinline__ bool dec_bar_and(bool v)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, 1, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v)
+        : "memory");
+    return r != 0;
+}
+
+// Store of a float to the shared memory of a CTA of the cluster (a
+// shared::cluster address from mapa_shared).
+__device__ __forceinline__ void st_dsmem_f32(uint32_t cluster_addr, float v)
+{
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(cluster_addr), "f"(v) : "memory");
+}
+
+// Bounded wait for the phase of `bar` with the given parity; false (and the
+// device status set) when the limit passed.
+__device__ __forceinline__ bool dec_wait(uint32_t bar, uint32_t parity)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > kDecWaitLimitNs) {
+            record_timeout();
+            return false;
+        }
+    }
+    return true;
+}
+
 // Power of two 2^e that brings max|x| (> 0) into [2^14, 2^15): hi parts then
 // stay far from fp16 overflow and lo parts keep 11 more bits.  Built from the
 // exponent bits, so 2^e and its inverse are exact; 1 for a zero maximum.
@@ -211,15 +270,15 @@ kv_decode_tc_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
     uint8_t *vtile = smem + S::kVTileOff;
     uint8_t *bq = smem + S::kBqOff;
     uint8_t *bw = smem + S::kBwOff;
-    const uint32_t bar_s = smem_u32(smem + S::kMiscOff);
+    const uint32_t bar_s = smem_u32(smem + S::kMiscOff);          // score MMAs done
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + S::kMiscOff + 8);
     const uint32_t bar_drain = smem_u32(smem + S::kMiscOff + 16);
-    const uint32_t bar_o = smem_u32(smem + S::kMiscOff + 24);
+    const uint32_t bar_o = smem_u32(smem + S::kMiscOff + 24);     // value MMAs done
+    const uint32_t bar_k = smem_u32(smem + S::kMiscOff + 32);     // key tile and B_q ready
+    const uint32_t bar_v = smem_u32(smem + S::kMiscOff + 40);     // value tile, B_w, D_o ready
+    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + S::kMiscOff + 48);
     float *red = reinterpret_cast<float *>(smem + S::kRedOff);      // [4][G + 1]
-    float *sm_m = reinterpret_cast<float *>(smem + S::kMOff);
-    float *sm_l = reinterpret_cast<float *>(smem + S::kLOff);
     float *lpart = reinterpret_cast<float *>(smem + S::kLpOff);     // [4][G]
-    float *fin = reinterpret_cast<float *>(smem + S::kFinOff);      // [G][128]
     float *inv_qs = reinterpret_cast<float *>(smem + S::kIqOff);    // [G]
     float *vmx = reinterpret_cast<float *>(smem + S::kVmOff);       // [4]
 
@@ -229,6 +288,7 @@ kv_decode_tc_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
     const int64_t b = blockIdx.z;
     const int Hq = Hkv * G;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool compute = warp < kDecCompute / 32;
     const float kInvSqrtD = 0.08838834764831845f;
     // softmax in base 2: scores / sqrt(128) times log2(e), then exp2
     const float kScoreMul = 0.08838834764831845f * 1.4426950408889634f;
@@ -236,11 +296,15 @@ kv_decode_tc_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
     const int64_t ts = min(T, (int64_t)r * slice);
     const int64_t te = min(T, ts + slice);
     const int ntiles = (int)((te - ts + kDecTile - 1) / kDecTile);
+    const int n_own = (G + nsplit - 1) / nsplit;       // heads this CTA finishes: r, r + nsplit, ...
 
     if (tid == 0) {
         mbar_init(bar_s, 1);
         mbar_init(bar_o, 1);
         mbar_init(bar_drain, 1);
+        mbar_init(bar_k, kDecCompute);
+        mbar_init(bar_v, kDecCompute);
+        *abort_flag = 0u;
         mbar_fence_init();
     }
     if (warp == 0) {
@@ -263,12 +327,11 @@ kv_decode_tc_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
         }
     };
     uint4 krow[4], vrow[4];
-    load_row(kq, 0, krow);
-    load_row(vq, 0, vrow);
-
-    // ---- the slice's largest value scale (the weights e * vs never exceed
-    // it, so one power-of-two scale serves every tile of the slice)
-    {
+    if (compute) {
+        load_row(kq, 0, krow);
+        load_row(vq, 0, vrow);
+        // ---- the slice's largest value scale (the weights e * vs never
+        // exceed it, so one power-of-two scale serves every tile of the slice)
         float vm = 0.f;
 #pragma unroll 4
         for (int j = 0; j < ntiles; ++j) {
@@ -279,305 +342,320 @@ kv_decode_tc_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
         vm = warp_max(vm, 32);
         if (lane == 0)
             vmx[warp] = vm;
-    }
-    // ---- rotate the G queries (16 threads per query, 8 elements each: bits
-    // 0-2 in registers, bits 3-6 through half-warp shuffles), as in the
-    // decode-scores kernel; the 16 threads of a query then find its maximum
-    // and write its hi / lo rows of B_q in the converted dim order
-    {
-        const int p = tid & 15;
-        const int8_t *sg = signs + h * 128 + 8 * p;
-#pragma unroll
-        for (int g0 = 0; g0 < G; g0 += kDecThreads / 16) {
-            const int g = g0 + (tid >> 4);
-            const bool gv = G % (kDecThreads / 16) == 0 || g < G;
-            const uint4 raw = gv ? *reinterpret_cast<const uint4 *>(q + (b * Hq + (int64_t)h * G + g) * 128 + 8 * p)
-                                 : make_uint4(0u, 0u, 0u, 0u);
-            const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-            float v[8];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float2 f = half2_bits_to_float2(w4[k]);
-                v[2 * k] = sg[2 * k] < 0 ? -f.x : f.x;
-                v[2 * k + 1] = sg[2 * k + 1] < 0 ? -f.y : f.y;
-            }
-#pragma unroll
-            for (int hb = 1; hb < 8; hb <<= 1)
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    if ((i & hb) == 0) {
-                        const float a = v[i], c = v[i + hb];
-                        v[i] = a + c;
-                        v[i + hb] = a - c;
+        // ---- rotate the G queries (16 threads per query, 8 elements each: bits
+        // 0-2 in registers, bits 3-6 through half-warp shuffles), as in the
+        // decode-scores kernel; the 16 threads of a query then find its maximum
+        // and write its hi / lo rows of B_q in the converted dim order
+        {
+            const int p = tid & 15;
+            const int8_t *sg = signs + h * 128 + 8 * p;
+    #pragma unroll
+            for (int g0 = 0; g0 < G; g0 += kDecCompute / 16) {
+                const int g = g0 + (tid >> 4);
+                const bool gv = G % (kDecCompute / 16) == 0 || g < G;
+                const uint4 raw = gv ? *reinterpret_cast<const uint4 *>(q + (b * Hq + (int64_t)h * G + g) * 128 + 8 * p)
+                                     : make_uint4(0u, 0u, 0u, 0u);
+                const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+                float v[8];
+    #pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float2 f = half2_bits_to_float2(w4[k]);
+                    v[2 * k] = sg[2 * k] < 0 ? -f.x : f.x;
+                    v[2 * k + 1] = sg[2 * k + 1] < 0 ? -f.y : f.y;
+                }
+    #pragma unroll
+                for (int hb = 1; hb < 8; hb <<= 1)
+    #pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        if ((i & hb) == 0) {
+                            const float a = v[i], c = v[i + hb];
+                            v[i] = a + c;
+                            v[i + hb] = a - c;
+                        }
+    #pragma unroll
+                for (int lb = 1; lb < 16; lb <<= 1) {
+                    const bool upper = (p & lb) != 0;
+    #pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float o = __shfl_xor_sync(0xffffffffu, v[i], lb);
+                        v[i] = upper ? o - v[i] : v[i] + o;
                     }
-#pragma unroll
-            for (int lb = 1; lb < 16; lb <<= 1) {
-                const bool upper = (p & lb) != 0;
-#pragma unroll
+                }
+                float mx = 0.f;
+    #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const float o = __shfl_xor_sync(0xffffffffu, v[i], lb);
-                    v[i] = upper ? o - v[i] : v[i] + o;
+                    v[i] *= kInvSqrtD;
+                    mx = fmaxf(mx, fabsf(v[i]));
+                }
+    #pragma unroll
+                for (int lb = 1; lb < 16; lb <<= 1)
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, lb));
+                float inv;
+                const float sc = dec_pow2_scale(mx, inv);
+                if (gv) {
+    #pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        dec_put_split<G>(bq, g, 8 * p + dec_dim(i), v[i] * sc);
+                    if (p == 0)
+                        inv_qs[g] = inv;
                 }
             }
-            float mx = 0.f;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                v[i] *= kInvSqrtD;
-                mx = fmaxf(mx, fabsf(v[i]));
-            }
-#pragma unroll
-            for (int lb = 1; lb < 16; lb <<= 1)
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, lb));
-            float inv;
-            const float sc = dec_pow2_scale(mx, inv);
-            if (gv) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    dec_put_split<G>(bq, g, 8 * p + dec_dim(i), v[i] * sc);
-                if (p == 0)
-                    inv_qs[g] = inv;
-            }
         }
-    }
-    if (tid < G) {
-        sm_m[tid] = -INFINITY;
-        sm_l[tid] = 0.f;
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    float inv_wsc;
-    const float wsc = dec_pow2_scale(fmaxf(fmaxf(vmx[0], vmx[1]), fmaxf(vmx[2], vmx[3])), inv_wsc);
-    float inv_q[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-        inv_q[g] = inv_qs[g];
     const uint32_t tmem = *tmem_slot;
-    const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
 
-    float lsum[G];                                    // this thread's share of sum exp2
+    if (!compute) {
+        // ---- warp 4: the MMAs of every tile, each once its operands are in
+        // place (lane 0 issues; the warp waits together)
+        constexpr uint32_t idesc_s = idesc_f16(128, NP);
+        constexpr uint32_t idesc_o = idesc_f16(128, NP) | (1u << 15);    // A (values) MN-major
+#pragma unroll 1
+        for (int j = 0; j < ntiles; ++j) {
+            if (!dec_wait(bar_k, j & 1) || *abort_flag)
+                break;
+            tc_fence_after();
+            if (lane == 0) {
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_f16_ss(tmem, desc_kmajor_sw128(smem_u32(ktile) + 16384 * (kk >> 2) + 32 * (kk & 3)),
+                                desc_kmajor_sw128(smem_u32(bq) + NP * 128 * (kk >> 2) + 32 * (kk & 3)), idesc_s,
+                                kk > 0 ? 1u : 0u);
+                umma_commit(bar_s);
+            }
+            __syncwarp();
+            if (!dec_wait(bar_v, j & 1) || *abort_flag)
+                break;
+            tc_fence_after();
+            if (lane == 0) {
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_f16_ss(tmem + NP, desc_mnmajor_sw128(smem_u32(vtile) + 2048 * kk, 16384),
+                                desc_kmajor_sw128(smem_u32(bw) + NP * 128 * (kk >> 2) + 32 * (kk & 3)), idesc_o,
+                                (j > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(bar_o);
+            }
+            __syncwarp();
+        }
+    }
+
+    float inv_wsc = 1.0f;
     float m_run[G];                                   // running maximum (base-2 units)
+    float lsum[G];                                    // this thread's share of sum exp2
+    uint32_t dout[NP];                                // the CTA's value accumulator, lane = dim
 #pragma unroll
     for (int g = 0; g < G; ++g) {
         lsum[g] = 0.f;
         m_run[g] = -INFINITY;
     }
-    uint32_t commits_s = 0, commits_o = 0;
     bool ok = true;
-    constexpr uint32_t idesc_s = idesc_f16(128, NP);
-    constexpr uint32_t idesc_o = idesc_f16(128, NP) | (1u << 15);    // A (values) MN-major
-    auto mma_wait = [&](uint32_t bar, uint32_t commits) {
-        // the latest commit to `bar` has completed (bounded; the CTA then gives up as a whole)
-        bool done = true;
-        if (!mbar_try_wait(bar, (commits - 1) & 1)) {
-            const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(bar, (commits - 1) & 1)) {
-                if (globaltimer_ns() - t0 > kDecWaitLimitNs) {
-                    record_timeout();
-                    done = false;
-                    break;
+    if (compute) {
+        const float wsc = dec_pow2_scale(fmaxf(fmaxf(vmx[0], vmx[1]), fmaxf(vmx[2], vmx[3])), inv_wsc);
+        float inv_q[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+            inv_q[g] = inv_qs[g];
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
+        // the latest commit to `bar` has completed, for every compute thread
+        auto wait_all = [&](uint32_t bar, int phase) { return dec_bar_and(dec_wait(bar, phase & 1)); };
+        // scales of token t of tile j (loaded one tile ahead)
+        auto load_scales = [&](int j, float &ksv, float &vsv) {
+            const int64_t t = ts + (int64_t)j * kDecTile + tid;
+            const bool tv = j < ntiles && t < te;
+            ksv = tv ? __half2float(ks[(b * T + t) * Hkv + h]) : 0.f;
+            vsv = tv ? __half2float(vs[(b * T + t) * Hkv + h]) : 0.f;
+        };
+        float ks_next, vs_next;
+        load_scales(0, ks_next, vs_next);
+        // Per tile j: keys converted -> (warp 4 issues the score MMAs) ->
+        // (value MMAs of tile j - 1 done) values converted while the score
+        // MMAs run -> scores, softmax weights -> (warp 4 issues the value
+        // MMAs, which run while the next tile's keys are converted).  The
+        // key tile is free at the top of an iteration: its MMAs were waited
+        // for before the scores were read.
+#pragma unroll 1
+        for (int j = 0; j < ntiles; ++j) {
+            const int64_t t = ts + (int64_t)j * kDecTile + tid;
+            const bool tv = t < te;
+            const float ksv = ks_next, vsv = vs_next;
+            load_scales(j + 1, ks_next, vs_next);
+            // ---- keys: convert, hand to the MMA warp
+            dec_convert_row(krow, ktile, tid);
+            load_row(kq, j + 1, krow);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar_k);
+            // ---- values: the previous tile's value MMAs are done with the
+            // value tile, B_w and D_o; convert while the score MMAs run
+            if (j > 0 && !(ok = wait_all(bar_o, j - 1)))
+                break;
+            dec_convert_row(vrow, vtile, tid);
+            load_row(vq, j + 1, vrow);
+            if (!(ok = wait_all(bar_s, j)))
+                break;
+            tc_fence_after();
+            // ---- scores of token t (lane t of D_s), the tile maxima
+            float sc[G];
+            {
+                uint32_t d[NP];
+                if constexpr (NP == 16) {
+                    uint32_t (&d16)[16] = *reinterpret_cast<uint32_t (*)[16]>(d);
+                    tmem_ld16(lane_base, d16);
+                    tmem_wait_ld16(d16);
+                } else {
+                    uint32_t (&d32)[32] = *reinterpret_cast<uint32_t (*)[32]>(d);
+                    tmem_ld32(lane_base, d32);
+                    tmem_wait_ld(d32);
+                }
+                // score / sqrt(128) in base-2 units: (hi + lo 2^-11) 2^-e ks / sqrt(128) log2(e)
+                const float km = ksv * kScoreMul;
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float x = (__uint_as_float(d[g]) + __uint_as_float(d[G + g]) * (1.0f / 2048.0f)) * inv_q[g];
+                    sc[g] = tv ? x * km : -INFINITY;
                 }
             }
-        }
-        return __syncthreads_and(done) != 0;
-    };
-
-    // scales of token t of tile j (loaded one tile ahead)
-    auto load_scales = [&](int j, float &ksv, float &vsv) {
-        const int64_t t = ts + (int64_t)j * kDecTile + tid;
-        const bool tv = j < ntiles && t < te;
-        ksv = tv ? __half2float(ks[(b * T + t) * Hkv + h]) : 0.f;
-        vsv = tv ? __half2float(vs[(b * T + t) * Hkv + h]) : 0.f;
-    };
-    float ks_next, vs_next;
-    load_scales(0, ks_next, vs_next);
-    // Per tile j: keys converted -> score MMAs issued -> (value MMAs of tile
-    // j - 1 done) values converted while the score MMAs run -> scores, softmax
-    // weights -> value MMAs issued, running while the next tile's keys are
-    // converted.  The key tile is free at the top of an iteration (its MMAs
-    // were waited for before the scores were read).
-#pragma unroll 1
-    for (int j = 0; j < ntiles && ok; ++j) {
-        const int64_t t = ts + (int64_t)j * kDecTile + tid;
-        const bool tv = t < te;
-        const float ksv = ks_next, vsv = vs_next;
-        load_scales(j + 1, ks_next, vs_next);
-        // ---- keys: convert, multiply with the query rows
-        dec_convert_row(krow, ktile, tid);
-        load_row(kq, j + 1, krow);
-        fence_proxy_async_smem();
-        __syncthreads();
-        if (tid == 0) {
-            tc_fence_after();
+            dec_tile_max<G>(sc, red + warp * (G + 1), lane);
+            dec_bar_sync();
+            // ---- softmax: all tile maxima first, then the arithmetic, then
+            // the stores of the weights (so that no load waits behind a store)
+            float tmax[G];
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                umma_f16_ss(tmem, desc_kmajor_sw128(smem_u32(ktile) + 16384 * (kk >> 2) + 32 * (kk & 3)),
-                            desc_kmajor_sw128(smem_u32(bq) + NP * 128 * (kk >> 2) + 32 * (kk & 3)), idesc_s,
-                            kk > 0 ? 1u : 0u);
-            umma_commit(bar_s);
-        }
-        ++commits_s;
-        // ---- values: the previous tile's value MMAs are done with the value
-        // tile and B_w; convert while the score MMAs run
-        if (j > 0 && !(ok = mma_wait(bar_o, commits_o)))
-            break;
-        dec_convert_row(vrow, vtile, tid);
-        load_row(vq, j + 1, vrow);
-        if (!(ok = mma_wait(bar_s, commits_s)))
-            break;
-        tc_fence_after();
-        // ---- scores of token t (lane t of D_s), the tile maxima
-        float s[G];
-        {
-            uint32_t d[NP];
-            if constexpr (NP == 16) {
-                uint32_t (&d16)[16] = *reinterpret_cast<uint32_t (*)[16]>(d);
-                tmem_ld16(lane_base, d16);
-                tmem_wait_ld16(d16);
-            } else {
-                uint32_t (&d32)[32] = *reinterpret_cast<uint32_t (*)[32]>(d);
-                tmem_ld32(lane_base, d32);
-                tmem_wait_ld(d32);
-            }
-            // score / sqrt(128) in base-2 units: (hi + lo 2^-11) 2^-e ks / sqrt(128) log2(e)
-            const float km = ksv * kScoreMul;
+            for (int g = 0; g < G; ++g)
+                tmax[g] = fmaxf(fmaxf(red[g], red[(G + 1) + g]), fmaxf(red[2 * (G + 1) + g], red[3 * (G + 1) + g]));
+            float beta[G], wgt[G];                    // rescale of the value accumulator, weights
+            bool rescale = false;
 #pragma unroll
             for (int g = 0; g < G; ++g) {
-                const float x = (__uint_as_float(d[g]) + __uint_as_float(d[G + g]) * (1.0f / 2048.0f)) * inv_q[g];
-                s[g] = tv ? x * km : -INFINITY;
+                const float m_new = fmaxf(m_run[g], tmax[g]);
+                const float alpha = m_run[g] == -INFINITY ? 0.f : dec_exp2(m_run[g] - m_new);
+                beta[g] = alpha;
+                rescale |= j > 0 && alpha != 1.0f;
+                const float e = tv ? dec_exp2(sc[g] - m_new) : 0.f;
+                lsum[g] = lsum[g] * alpha + e;
+                m_run[g] = m_new;
+                wgt[g] = e * vsv * wsc;
             }
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+                dec_put_split<G>(bw, g, tid, wgt[g]);
+            // the value accumulator in the units of this tile (lane = dim)
+            if (rescale) {
+                uint32_t d[NP];
+                if constexpr (NP == 16) {
+                    uint32_t (&d16)[16] = *reinterpret_cast<uint32_t (*)[16]>(d);
+                    tmem_ld16(lane_base + NP, d16);
+                    tmem_wait_ld16(d16);
+                } else {
+                    uint32_t (&d32)[32] = *reinterpret_cast<uint32_t (*)[32]>(d);
+                    tmem_ld32(lane_base + NP, d32);
+                    tmem_wait_ld(d32);
+                }
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    d[g] = __float_as_uint(__uint_as_float(d[g]) * beta[g]);
+                    d[G + g] = __float_as_uint(__uint_as_float(d[G + g]) * beta[g]);
+                }
+                if constexpr (NP == 16)
+                    tmem_st16(lane_base + NP, *reinterpret_cast<uint32_t (*)[16]>(d));
+                else
+                    tmem_st32(lane_base + NP, *reinterpret_cast<uint32_t (*)[32]>(d));
+                tmem_wait_st();
+            }
+            // ---- hand the value tile, B_w and D_o to the MMA warp
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar_v);
         }
-        dec_tile_max<G>(s, red + warp * (G + 1), lane);
-        __syncthreads();
-        float beta[G];                               // rescale of the value accumulator
-        bool rescale = false;
+        if (!ok) {
+            // the MMA warp may wait for this tile's values: release it
+            *abort_flag = 1u;
+            mbar_arrive(bar_v);
+        }
+        if (ok && ntiles > 0)
+            ok = wait_all(bar_o, ntiles - 1);
+        // ---- this CTA's partial result: the accumulator (lane = dim), m, l
+        if (ok && ntiles > 0) {
+            tc_fence_after();
+            if constexpr (NP == 16) {
+                tmem_ld16(lane_base + NP, *reinterpret_cast<uint32_t (*)[16]>(dout));
+                tmem_wait_ld16(*reinterpret_cast<uint32_t (*)[16]>(dout));
+            } else {
+                tmem_ld32(lane_base + NP, *reinterpret_cast<uint32_t (*)[32]>(dout));
+                tmem_wait_ld(*reinterpret_cast<uint32_t (*)[32]>(dout));
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < NP; ++i)
+                dout[i] = 0u;
+        }
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-            const float tmax = fmaxf(fmaxf(red[g], red[(G + 1) + g]), fmaxf(red[2 * (G + 1) + g], red[3 * (G + 1) + g]));
-            const float m_new = fmaxf(m_run[g], tmax);
-            const float alpha = m_run[g] == -INFINITY ? 0.f : exp2f(m_run[g] - m_new);
-            beta[g] = alpha;
-            rescale |= j > 0 && alpha != 1.0f;
-            const float e = tv ? exp2f(s[g] - m_new) : 0.f;
-            lsum[g] = lsum[g] * alpha + e;
-            m_run[g] = m_new;
-            dec_put_split<G>(bw, g, tid, e * vsv * wsc);
+            const float ls = warp_sum_f(lsum[g]);
+            if (lane == 0)
+                lpart[warp * G + g] = ls;
         }
-        // the value accumulator in the units of this tile (lane = dim)
-        if (rescale) {
-            uint32_t d[NP];
-            if constexpr (NP == 16) {
-                uint32_t (&d16)[16] = *reinterpret_cast<uint32_t (*)[16]>(d);
-                tmem_ld16(lane_base + NP, d16);
-                tmem_wait_ld16(d16);
-            } else {
-                uint32_t (&d32)[32] = *reinterpret_cast<uint32_t (*)[32]>(d);
-                tmem_ld32(lane_base + NP, d32);
-                tmem_wait_ld(d32);
-            }
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                d[g] = __float_as_uint(__uint_as_float(d[g]) * beta[g]);
-                d[G + g] = __float_as_uint(__uint_as_float(d[G + g]) * beta[g]);
-            }
-            if constexpr (NP == 16)
-                tmem_st16(lane_base + NP, *reinterpret_cast<uint32_t (*)[16]>(d));
-            else
-                tmem_st32(lane_base + NP, *reinterpret_cast<uint32_t (*)[32]>(d));
-            tmem_wait_st();
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                umma_f16_ss(tmem + NP, desc_mnmajor_sw128(smem_u32(vtile) + 2048 * kk, 16384),
-                            desc_kmajor_sw128(smem_u32(bw) + NP * 128 * (kk >> 2) + 32 * (kk & 3)), idesc_o,
-                            (j > 0 || kk > 0) ? 1u : 0u);
-            umma_commit(bar_o);
-        }
-        ++commits_o;
-    }
-    if (ok && ntiles > 0)
-        ok = mma_wait(bar_o, commits_o);
-
-    // ---- this CTA's partial result: fin[g][d] (unnormalized), m, l
-    if (ok && ntiles > 0) {
-        tc_fence_after();
-        uint32_t d[NP];
-        if constexpr (NP == 16) {
-            uint32_t (&d16)[16] = *reinterpret_cast<uint32_t (*)[16]>(d);
-            tmem_ld16(lane_base + NP, d16);
-            tmem_wait_ld16(d16);
-        } else {
-            uint32_t (&d32)[32] = *reinterpret_cast<uint32_t (*)[32]>(d);
-            tmem_ld32(lane_base + NP, d32);
-            tmem_wait_ld(d32);
-        }
-        const int dim = dec_dim(tid);
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-            fin[g * 128 + dim] = (__uint_as_float(d[g]) + __uint_as_float(d[G + g]) * (1.0f / 2048.0f)) * inv_wsc;
-    } else {
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-            fin[g * 128 + tid] = 0.f;
-    }
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        const float ls = warp_sum_f(lsum[g]);
-        if (lane == 0)
-            lpart[warp * G + g] = ls;
-    }
-    __syncthreads();
-    if (tid < G) {
-        sm_l[tid] = ntiles > 0 ? (lpart[tid] + lpart[G + tid]) + (lpart[2 * G + tid] + lpart[3 * G + tid]) : 0.f;
-        sm_m[tid] = ntiles > 0 ? m_run[tid] : -INFINITY;
+        dec_bar_sync();
     }
 
-    // combine the slices of the cluster: CTA r finishes heads r, r + S, ...
+    // ---- combine the slices of the cluster.  After the first cluster
+    // barrier every CTA's loop is over and its value tile free; each CTA then
+    // stores its partial result for head g into the value tile of the CTA
+    // that finishes g (rank g mod nsplit, slot g div nsplit); after the
+    // second barrier each CTA combines what it received:
+    // out = sum_r exp2(m_r - M) acc_r / sum_r exp2(m_r - M) l_r, M = max_r m_r.
+    float *recv = reinterpret_cast<float *>(smem + S::kRecvOff);         // [nsplit][n_own][128]
+    float *recv_ml = reinterpret_cast<float *>(smem + S::kRecvMlOff);    // [2][nsplit][n_own]
     cluster_sync_all();
-    const uint32_t a_fin = smem_u32(fin);
-    const uint32_t a_m = smem_u32(sm_m);
-    const uint32_t a_l = smem_u32(sm_l);
-    for (int g = r; g < G; g += nsplit) {
-        float mq[kDecMaxSplit], lq[kDecMaxSplit], fq[kDecMaxSplit];
+    if (compute) {
+        const int dim = dec_dim(tid);
+        const bool have = ok && ntiles > 0;
 #pragma unroll
-        for (int qq = 0; qq < kDecMaxSplit; ++qq) {
-            if (qq < nsplit) {
-                mq[qq] = ld_dsmem_f32(mapa_shared(a_m + 4 * g, qq));
-                lq[qq] = ld_dsmem_f32(mapa_shared(a_l + 4 * g, qq));
-                fq[qq] = ld_dsmem_f32(mapa_shared(a_fin + 4 * (g * 128 + tid), qq));
-            } else {
-                mq[qq] = -INFINITY;
-                lq[qq] = 0.f;
-                fq[qq] = 0.f;
+        for (int g = 0; g < G; ++g) {
+            const int owner = g % nsplit, slot = g / nsplit;
+            const float v = (__uint_as_float(dout[g]) + __uint_as_float(dout[G + g]) * (1.0f / 2048.0f)) * inv_wsc;
+            st_dsmem_f32(mapa_shared(smem_u32(recv + (r * n_own + slot) * 128 + dim), owner), v);
+        }
+        if (tid < G) {
+            const int g = tid, owner = g % nsplit, slot = g / nsplit;
+            const float l = have ? (lpart[g] + lpart[G + g]) + (lpart[2 * G + g] + lpart[3 * G + g]) : 0.f;
+            float m = -INFINITY;                     // m_run[g], selected without indexing by a variable
+#pragma unroll
+            for (int i = 0; i < G; ++i)
+                m = (have && i == g) ? m_run[i] : m;
+            st_dsmem_f32(mapa_shared(smem_u32(recv_ml + r * n_own + slot), owner), m);
+            st_dsmem_f32(mapa_shared(smem_u32(recv_ml + nsplit * n_own + r * n_own + slot), owner), l);
+        }
+    }
+    cluster_sync_all();
+    if (compute) {
+        for (int slot = 0; slot < n_own; ++slot) {
+            const int g = r + slot * nsplit;
+            if (g >= G)
+                break;
+            float M = -INFINITY;
+            for (int qq = 0; qq < nsplit; ++qq)
+                M = fmaxf(M, recv_ml[qq * n_own + slot]);
+            float num = 0.f, den = 0.f;
+            for (int qq = 0; qq < nsplit; ++qq) {
+                const float mq = recv_ml[qq * n_own + slot];
+                const float f = mq == -INFINITY ? 0.f : exp2f(mq - M);
+                den = fmaf(f, recv_ml[nsplit * n_own + qq * n_own + slot], den);
+                num = fmaf(f, recv[(qq * n_own + slot) * 128 + tid], num);
             }
+            out[(b * Hq + (int64_t)h * G + g) * 128 + tid] = num / den;
         }
-        float M = -INFINITY;
-#pragma unroll
-        for (int qq = 0; qq < kDecMaxSplit; ++qq)
-            M = fmaxf(M, mq[qq]);
-        float num = 0.f, den = 0.f;
-#pragma unroll
-        for (int qq = 0; qq < kDecMaxSplit; ++qq) {
-            const float f = mq[qq] == -INFINITY ? 0.f : exp2f(mq[qq] - M);
-            den = fmaf(f, lq[qq], den);
-            num = fmaf(f, fq[qq], num);
-        }
-        out[(b * Hq + (int64_t)h * G + g) * 128 + tid] = num / den;
     }
     // every MMA this CTA issued has completed (also after a timeout)
-    if (tid == 0) {
+    if (warp == kDecCompute / 32 && lane == 0) {
         umma_commit(bar_drain);
         mbar_wait_drain(bar_drain, 0, kDecWaitLimitNs);
     }
     tc_fence_before();
     __syncthreads();
-    cluster_sync_all();                   // no CTA leaves while another may still read its memory
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, S::kTmemCols);

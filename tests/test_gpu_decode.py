@@ -17,9 +17,13 @@ perturbed by at most eps move by sum_t |dp_t| <= 2 eps / sqrt(128) in total,
 so the output moves by at most that times max_t |vs_t code_t|.  The value
 product itself is the attention tail's convex combination in fp32, bounded as
 in the test of quarot_kv_decode_attend by 4 (T + 32) 2^-24 max_t |vs_t code_t|
-(the weights' two-part fp16 split adds 2^-22 relative).  So
+(the weights' two-part fp16 split adds 2^-22 relative).  The weights come from
+the hardware base-2 exponential (ex2.approx, a few ulp): with each weight off
+by at most eps_x = 2^-21 relative, the normalized output moves by at most
+2 eps_x max_t |vs_t code_t| (the rescale factors' errors cancel between the
+accumulator and the sum of weights).  So
 
-    |out - ref| <= (4 (T + 32) 2^-24 + 2 eps_s / sqrt(128)) max_t |vs_t code_t|.
+    |out - ref| <= (4 (T + 32) 2^-24 + 2^-20 + 2 eps_s / sqrt(128)) max_t |vs_t code_t|.
 """
 import numpy as np
 import pytest
@@ -60,7 +64,7 @@ def _bound(qh, s, kq, ks, vq, vs):
     eps_s = 2.0 ** -15 * ksmax * 8.0 * qsum
     vmax = np.abs(oracle.unpack(vq).astype(np.float64) * oracle.f16_to_f64(vs)[..., None]).max(axis=(1, 3))
     vmax = np.repeat(vmax, G, axis=1)                                               # [B, Hq]
-    return ((4.0 * (T + 32) * 2.0 ** -24 + 2.0 * eps_s / np.sqrt(128.0)) * vmax)[..., None] + 1e-30
+    return ((4.0 * (T + 32) * 2.0 ** -24 + 2.0 ** -20 + 2.0 * eps_s / np.sqrt(128.0)) * vmax)[..., None] + 1e-30
 
 
 def _decode_check(q, qh, s, kq, ks, vq, vs):
