@@ -57,7 +57,9 @@ typedef enum {
     QUAROT_ERR_MISALIGNED = 3,       /* a pointer not 16-byte aligned */
     QUAROT_ERR_CUDA = 4,             /* the CUDA runtime reported an error */
     QUAROT_ERR_DEVICE_TIMEOUT = 5,   /* a kernel gave up a bounded wait (see below) */
-    QUAROT_ERR_NO_DEVICE = 6         /* no sm_100 device is current */
+    QUAROT_ERR_NO_DEVICE = 6,        /* no sm_100 device is current */
+    QUAROT_ERR_DEVICE_BOUNDS = 7     /* bounds-checking build only: a kernel skipped a store
+                                        outside its output (see quarot_debug_bounds) */
 } quarot_status_t;
 
 /* A cudaStream_t passed as an opaque pointer. */
@@ -463,8 +465,9 @@ quarot_status_t quarot_kv_decode_attention(const void *q_f16, int64_t Hq, const 
 /*
  * quarot_get_device_status -- synchronizes `stream` (the whole current device
  * when stream is NULL), then reports (and clears) the library's device-side
- * error word: QUAROT_ERR_DEVICE_TIMEOUT if any kernel since the last call
- * gave up a bounded wait (every wait on a barrier, a copy or the tensor core
+ * error word: QUAROT_ERR_DEVICE_BOUNDS if (bounds-checking build only) a
+ * kernel skipped a store outside its output, else QUAROT_ERR_DEVICE_TIMEOUT if
+ * any kernel since the last call gave up a bounded wait (every wait on a barrier, a copy or the tensor core
  * is bounded in time; on expiry the kernel records the fact, waits -- again
  * with a limit -- for the copies and tensor-core work it issued, frees its
  * tensor memory and exits), QUAROT_ERR_CUDA if the synchronization itself
@@ -515,6 +518,18 @@ quarot_status_t quarot_probe_mma_i8(int64_t steps, int operands, int64_t *pairs,
  */
 quarot_status_t quarot_test_wait_timeout(const void *v_f16, int64_t rows, uint8_t *q_packed, void *scales_f16,
                                          int64_t withheld_tile, uint64_t wait_limit_ns, quarot_stream_t stream);
+
+/*
+ * quarot_debug_bounds -- 1 for the bounds-checking build of the library
+ * (libquarot_dbg.so, compiled with QUAROT_DEBUG_BOUNDS), 0 for the normal
+ * one.  No passage of the pages corresponds to it: it is a test aid.  In the
+ * bounds-checking build every kernel checks, before each global store of an
+ * output, that the bytes it is about to write lie inside that output as the
+ * call's sizes give it; a store that would not is skipped and recorded, and
+ * quarot_get_device_status() then returns QUAROT_ERR_DEVICE_BOUNDS (before a
+ * timeout, if both happened).  The normal build has no such checks.
+ */
+int quarot_debug_bounds(void);
 
 /* Static, human-readable name of a status code. */
 const char *quarot_status_string(quarot_status_t status);

@@ -16,7 +16,11 @@ from typing import Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libquarot.so")
+# QUAROT_DEBUG_BOUNDS=1 in the environment selects the bounds-checking build
+# (libquarot_dbg.so: every kernel checks its output stores; see
+# quarot_debug_bounds in include/quarot.h)
+DEBUG_BOUNDS = os.environ.get("QUAROT_DEBUG_BOUNDS", "0") not in ("", "0")
+LIB_PATH = os.path.join(_HERE, "libquarot_dbg.so" if DEBUG_BOUNDS else "libquarot.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "quarot.h")
 
 if not os.path.exists(LIB_PATH):
@@ -56,6 +60,7 @@ _SIGS = {
     "quarot_get_device_status": ([_P], _INT),
     "quarot_status_string": ([_INT], ctypes.c_char_p),
     "quarot_last_error": ([], ctypes.c_char_p),
+    "quarot_debug_bounds": ([], _INT),
 }
 for _name, (_args, _ret) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -64,7 +69,7 @@ for _name, (_args, _ret) in _SIGS.items():
 
 STATUS = {0: "QUAROT_OK", 1: "QUAROT_ERR_INVALID_ARG", 2: "QUAROT_ERR_UNSUPPORTED_SHAPE",
           3: "QUAROT_ERR_MISALIGNED", 4: "QUAROT_ERR_CUDA", 5: "QUAROT_ERR_DEVICE_TIMEOUT",
-          6: "QUAROT_ERR_NO_DEVICE"}
+          6: "QUAROT_ERR_NO_DEVICE", 7: "QUAROT_ERR_DEVICE_BOUNDS"}
 
 
 class QuarotError(RuntimeError):

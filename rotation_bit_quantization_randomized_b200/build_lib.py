@@ -12,6 +12,9 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libquarot.so")
+# the bounds-checking build: every kernel checks its output stores
+# (QUAROT_DEBUG_BOUNDS; see quarot_debug_bounds in include/quarot.h)
+LIB_DEBUG = os.path.join(PKG, "libquarot_dbg.so")
 SOURCES = [os.path.join(CSRC, "quarot_api.cu")]
 HEADERS = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + \
     [os.path.join(ROOT, "include", "quarot.h")]
@@ -31,24 +34,35 @@ def _nvcc():
     return p if os.path.exists(p) else "nvcc"
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(f) <= t for f in SOURCES + HEADERS)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
+def build(force: bool = False, verbose: bool = False, debug_bounds: bool = False) -> str:
+    lib = LIB_DEBUG if debug_bounds else LIB
+    if not force and up_to_date(lib):
+        return lib
     cmd = [_nvcc()] + NVCC_FLAGS + ["-I", os.path.join(ROOT, "include"), "-I", CSRC]
+    if debug_bounds:
+        cmd += ["-DQUAROT_DEBUG_BOUNDS"]
     if verbose:
         cmd += ["-Xptxas", "-v"]
-    cmd += ["-o", LIB + ".tmp"] + SOURCES
+    cmd += ["-o", lib + ".tmp"] + SOURCES
     subprocess.run(cmd, check=True)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
+
+
+def build_all(force: bool = False) -> None:
+    """The normal library and the bounds-checking one, compiled side by side."""
+    import concurrent.futures as cf
+    with cf.ThreadPoolExecutor(2) as ex:
+        for f in [ex.submit(build, force, False, False), ex.submit(build, force, False, True)]:
+            f.result()
 
 
 if __name__ == "__main__":
-    print(build(force=True, verbose="-v" in sys.argv))
+    print(build(force=True, verbose="-v" in sys.argv, debug_bounds="--debug-bounds" in sys.argv))

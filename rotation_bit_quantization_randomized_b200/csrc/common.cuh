@@ -7,13 +7,35 @@
 
 namespace quarot {
 
-// Device-side error word: set when a bounded wait in a kernel expires.
-// Read and cleared on the host by quarot_get_device_status().
+// Device-side error word, one bit per kind of failure: a bounded wait in a
+// kernel expired, or (bounds-checking builds only) a store fell outside its
+// output.  Read and cleared on the host by quarot_get_device_status().
 __device__ int g_device_status;
 
-enum : int { kDevOk = 0, kDevTimeout = 1 };
+enum : int { kDevOk = 0, kDevTimeout = 1, kDevBounds = 2 };
 
-__device__ __forceinline__ void record_timeout() { atomicExch(&g_device_status, kDevTimeout); }
+__device__ __forceinline__ void record_timeout() { atomicOr(&g_device_status, kDevTimeout); }
+
+// Bounds-checking builds (QUAROT_DEBUG_BOUNDS defined): before each global
+// store of an output, QUAROT_IN_RANGE(p, bytes, base, total) checks that the
+// `bytes` written at p lie inside the output [base, base + total) as the
+// kernel's size arguments give it; on failure it sets the bounds bit of the
+// device status word and yields false, so that the store is skipped.  In
+// normal builds it is the constant true and its arguments are not evaluated.
+#ifdef QUAROT_DEBUG_BOUNDS
+__device__ __forceinline__ bool debug_in_range(const void *p, size_t bytes, const void *base, size_t total)
+{
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p), b = reinterpret_cast<uintptr_t>(base);
+    const bool ok = a >= b && a + bytes <= b + total;
+    if (!ok)
+        atomicOr(&g_device_status, kDevBounds);
+    return ok;
+}
+#define QUAROT_IN_RANGE(p, bytes, base, total) \
+    (::quarot::debug_in_range((const void *)(p), (size_t)(bytes), (const void *)(base), (size_t)(total)))
+#else
+#define QUAROT_IN_RANGE(p, bytes, base, total) (true)
+#endif
 
 __device__ __forceinline__ uint64_t globaltimer_ns()
 {

@@ -262,7 +262,8 @@ int8_gemm_pair_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_
                                 const float f1 = __int2float_rn((int)r[8 * v + 2 * i + 1]) * sam * wv[2 * i + 1];
                                 h[i] = h2_as_u32(__floats2half2_rn(f0, f1));
                             }
-                            *reinterpret_cast<uint4 *>(orow + n) = make_uint4(h[0], h[1], h[2], h[3]);
+                            if (QUAROT_IN_RANGE(orow + n, 16, a.out, a.M * a.N * 2))
+                                *reinterpret_cast<uint4 *>(orow + n) = make_uint4(h[0], h[1], h[2], h[3]);
                         }
                     }
                 } else if (mrow) {
@@ -270,7 +271,7 @@ int8_gemm_pair_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_
 #pragma unroll
                     for (int v = 0; v < 8; ++v) {
                         const int64_t n = n0 + 32 * c + 4 * v;
-                        if (n < a.N)
+                        if (n < a.N && QUAROT_IN_RANGE(orow + n, 16, a.out, a.M * a.N * 4))
                             *reinterpret_cast<int4 *>(orow + n) =
                                 make_int4((int)r[4 * v], (int)r[4 * v + 1], (int)r[4 * v + 2], (int)r[4 * v + 3]);
                     }

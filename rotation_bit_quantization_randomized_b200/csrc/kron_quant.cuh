@@ -449,8 +449,9 @@ kron_quant_kernel(const __grid_constant__ CUtensorMap tma_h,     // H^T, fp16 [3
                     const float a = fmaxf(fmaxf(red[(4 * h) * 2 + k], red[(4 * h + 1) * 2 + k]),
                                           fmaxf(red[(4 * h + 2) * 2 + k], red[(4 * h + 3) * 2 + k]));
                     rr[k] = a > 0.f ? 7.0f / a : 0.f;
-                    if (wq == 0 && lane == 0 && row0 + rbase + k < M)
-                        reinterpret_cast<float *>(scales)[row0 + rbase + k] = a * scale_mul;
+                    float *sdst = reinterpret_cast<float *>(scales) + row0 + rbase + k;
+                    if (wq == 0 && lane == 0 && row0 + rbase + k < M && QUAROT_IN_RANGE(sdst, 4, scales, M * 4))
+                        *sdst = a * scale_mul;
                 }
                 epi_barrier_and(kEpiThreads, true);      // red is free for the next tile
             }
@@ -494,12 +495,15 @@ kron_quant_kernel(const __grid_constant__ CUtensorMap tma_h,     // H^T, fp16 [3
                         gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 2));
                         __half s16;
                         rq = group_scale(gmax, scale_mul, sqrt_n, s16);
-                        if (rvalid && ap < kKronM && (lane & 3) == 0)
-                            reinterpret_cast<__half *>(scales)[row * (kKronK / 128) + ap / 4] = s16;
+                        __half *sdst = reinterpret_cast<__half *>(scales) + row * (kKronK / 128) + ap / 4;
+                        if (rvalid && ap < kKronM && (lane & 3) == 0 &&
+                            QUAROT_IN_RANGE(sdst, 2, scales, M * (kKronK / 128) * 2))
+                            *sdst = s16;
                     }
                     const uint4 pk = quant_pack32<GROUP>(v, rq);
-                    if (rvalid && ap < kKronM)
-                        *reinterpret_cast<uint4 *>(q + row * (kKronK / 2) + ap * 16) = pk;
+                    uint8_t *qdst = q + row * (kKronK / 2) + ap * 16;
+                    if (rvalid && ap < kKronM && QUAROT_IN_RANGE(qdst, 16, q, M * (kKronK / 2)))
+                        *reinterpret_cast<uint4 *>(qdst) = pk;
                 }
             }
         }

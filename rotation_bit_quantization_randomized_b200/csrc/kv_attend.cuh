@@ -250,7 +250,9 @@ kv_attend_kernel(const float *__restrict__ scores,    // [B, Hq, T]
             den = fmaf(f, lq[q], den);
             num = fmaf(f, fq[q], num);
         }
-        out[(b * Hq + (int64_t)h * G + g) * 128 + tid] = num / den;
+        float *dst = out + (b * Hq + (int64_t)h * G + g) * 128 + tid;
+        if (QUAROT_IN_RANGE(dst, 4, out, (int64_t)gridDim.z * Hq * 128 * 4))
+            *dst = num / den;
     }
     // no CTA leaves while another may still read its shared memory
     cluster_sync_all();

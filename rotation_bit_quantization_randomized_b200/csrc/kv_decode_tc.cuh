@@ -617,7 +617,9 @@ kv_decode_tc_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
         for (int g = 0; g < G; ++g) {
             const int owner = g % nsplit, slot = g / nsplit;
             const float v = (__uint_as_float(dout[g]) + __uint_as_float(dout[G + g]) * (1.0f / 2048.0f)) * inv_wsc;
-            st_dsmem_f32(mapa_shared(smem_u32(recv + (r * n_own + slot) * 128 + dim), owner), v);
+            float *slot_p = recv + (r * n_own + slot) * 128 + dim;
+            if (QUAROT_IN_RANGE(slot_p, 4, recv, S::kRecvMlOff - S::kRecvOff))
+                st_dsmem_f32(mapa_shared(smem_u32(slot_p), owner), v);
         }
         if (tid < G) {
             const int g = tid, owner = g % nsplit, slot = g / nsplit;
@@ -646,7 +648,9 @@ kv_decode_tc_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
                 den = fmaf(f, recv_ml[nsplit * n_own + qq * n_own + slot], den);
                 num = fmaf(f, recv[(qq * n_own + slot) * 128 + tid], num);
             }
-            out[(b * Hq + (int64_t)h * G + g) * 128 + tid] = num / den;
+            float *dst = out + (b * Hq + (int64_t)h * G + g) * 128 + tid;
+            if (QUAROT_IN_RANGE(dst, 4, out, (int64_t)gridDim.z * Hq * 128 * 4))
+                *dst = num / den;
         }
     }
     // every MMA this CTA issued has completed (also after a timeout)

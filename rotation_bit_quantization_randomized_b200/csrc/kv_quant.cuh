@@ -130,9 +130,10 @@ kv_quant_tma_kernel(const __grid_constant__ CUtensorMap tmap,   // fp16 [rows, 1
         const bool valid = row < rows;
         __half s16;
         const float r = group_scale(amax, scale_mul, sqrt_n, s16);
-        if (valid)
+        if (valid && QUAROT_IN_RANGE(scales + row, 2, scales, rows * 2))
             scales[row] = s16;
-        quant_pack_store<128>(v, r, q + (valid ? row : 0) * 64, valid, scale_needs_clamp(s16));
+        uint8_t *qdst = q + (valid ? row : 0) * 64;
+        quant_pack_store<128>(v, r, qdst, valid && QUAROT_IN_RANGE(qdst, 64, q, rows * 64), scale_needs_clamp(s16));
     }
     // copies issued beyond the consumed tiles (abort only) land before exit:
     // iterations it .. issued - 1 had their copies issued but were not waited for

@@ -158,8 +158,11 @@ kv_scores_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
         if (t < T) {
             const float s = __half2float(ks[(b * T + t) * Hkv + h]);
 #pragma unroll
-            for (int g = 0; g < G; ++g)
-                scores[(b * Hq + (int64_t)h * G + g) * T + t] = acc[i][g] * s;
+            for (int g = 0; g < G; ++g) {
+                float *dst = scores + (b * Hq + (int64_t)h * G + g) * T + t;
+                if (QUAROT_IN_RANGE(dst, 4, scores, (int64_t)gridDim.z * Hq * T * 4))
+                    *dst = acc[i][g] * s;
+            }
         }
     }
 }

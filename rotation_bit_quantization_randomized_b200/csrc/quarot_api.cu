@@ -1538,9 +1538,20 @@ quarot_status_t quarot_get_device_status(quarot_stream_t stream)
     if (v != kDevOk) {
         const int zero = 0;
         cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
+        if (v & kDevBounds)
+            return fail(QUAROT_ERR_DEVICE_BOUNDS, "a kernel skipped a store outside its output (bounds-checking build)");
         return fail(QUAROT_ERR_DEVICE_TIMEOUT, "a kernel gave up a bounded wait");
     }
     return QUAROT_OK;
+}
+
+int quarot_debug_bounds(void)
+{
+#ifdef QUAROT_DEBUG_BOUNDS
+    return 1;
+#else
+    return 0;
+#endif
 }
 
 const char *quarot_status_string(quarot_status_t status)
@@ -1552,6 +1563,7 @@ const char *quarot_status_string(quarot_status_t status)
     case QUAROT_ERR_MISALIGNED: return "QUAROT_ERR_MISALIGNED";
     case QUAROT_ERR_CUDA: return "QUAROT_ERR_CUDA";
     case QUAROT_ERR_DEVICE_TIMEOUT: return "QUAROT_ERR_DEVICE_TIMEOUT";
+    case QUAROT_ERR_DEVICE_BOUNDS: return "QUAROT_ERR_DEVICE_BOUNDS";
     case QUAROT_ERR_NO_DEVICE: return "QUAROT_ERR_NO_DEVICE";
     }
     return "QUAROT_ERR_UNKNOWN";

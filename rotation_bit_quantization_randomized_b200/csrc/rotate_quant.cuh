@@ -345,8 +345,9 @@ fwht_quant_kernel(const uint32_t *__restrict__ x,      // [M, K/2] fp16 pairs
             const float dv = (hi - lo) / 15.0f;
             const float z = dv > 0.f ? rintf(-lo / dv) : 0.f;
             const float r = dv > 0.f ? 1.0f / dv : 0.f;
-            uint32_t csum = quant_pack_store_asym(v, r, 12582912.0f + z, q + (valid ? row : 0) * (N / 2) + tr * 64,
-                                                  valid);
+            uint8_t *qdst = q + (valid ? row : 0) * (N / 2) + tr * 64;
+            uint32_t csum = quant_pack_store_asym(v, r, 12582912.0f + z, qdst,
+                                                  valid && QUAROT_IN_RANGE(qdst, 64, q, M * (N / 2)));
             if (T <= 32) {
                 csum = warp_sum(csum, T);
             } else {
@@ -356,7 +357,9 @@ fwht_quant_kernel(const uint32_t *__restrict__ x,      // [M, K/2] fp16 pairs
                 __syncthreads();
                 csum = reinterpret_cast<uint32_t *>(red)[4] + reinterpret_cast<uint32_t *>(red)[5];
             }
-            if (valid && tr == 0) {
+            if (valid && tr == 0 && QUAROT_IN_RANGE(reinterpret_cast<float *>(scales) + row, 4, scales, M * 4) &&
+                QUAROT_IN_RANGE(asym.zeros + row, 4, asym.zeros, M * 4) &&
+                QUAROT_IN_RANGE(asym.rowsums + row, 4, asym.rowsums, M * 4)) {
                 reinterpret_cast<float *>(scales)[row] = dv * scale_mul;
                 asym.zeros[row] = (int32_t)z;
                 asym.rowsums[row] = (int32_t)csum;
@@ -377,19 +380,23 @@ fwht_quant_kernel(const uint32_t *__restrict__ x,      // [M, K/2] fp16 pairs
                 amax = fmaxf(red[0], red[1]);
             }
             r = amax > 0.f ? kQmax / amax : 0.f;
-            if (valid && tr == 0)
+            if (valid && tr == 0 && QUAROT_IN_RANGE(reinterpret_cast<float *>(scales) + row, 4, scales, M * 4))
                 reinterpret_cast<float *>(scales)[row] = amax * scale_mul;
         } else {
             __syncthreads();
             __half s16;
             r = group_scale(amax, scale_mul, sqrt_n, s16);
-            if (valid)
-                reinterpret_cast<__half *>(scales)[row * (N / 128) + tr] = s16;
+            __half *sdst = reinterpret_cast<__half *>(scales) + row * (N / 128) + tr;
+            if (valid && QUAROT_IN_RANGE(sdst, 2, scales, M * (N / 128) * 2))
+                *sdst = s16;
         }
-        if (BITS != 4)
-            quant_store_i8(v, r, reinterpret_cast<int8_t *>(q) + (valid ? row : 0) * N + tr * 128, valid);
-        else
-            quant_pack_store<GROUP>(v, r, q + (valid ? row : 0) * (N / 2) + tr * 64, valid);
+        if (BITS != 4) {
+            int8_t *qdst = reinterpret_cast<int8_t *>(q) + (valid ? row : 0) * N + tr * 128;
+            quant_store_i8(v, r, qdst, valid && QUAROT_IN_RANGE(qdst, 128, q, M * N));
+        } else {
+            uint8_t *qdst = q + (valid ? row : 0) * (N / 2) + tr * 64;
+            quant_pack_store<GROUP>(v, r, qdst, valid && QUAROT_IN_RANGE(qdst, 64, q, M * (N / 2)));
+        }
     }
     // after an abort the copy of the iteration that was given up was issued
     // (in the previous iteration, or before the loop) and may still be in
@@ -497,9 +504,12 @@ block128_quant_kernel(const uint4 *__restrict__ x,     // [M, K] fp16, 8 per uin
                 const float amax = absmax128(v);
                 __half s16;
                 const float r = group_scale(amax, scale_mul, sqrt_n, s16);
-                if (ok)
-                    reinterpret_cast<__half *>(scales)[row * nb + b] = s16;
-                quant_pack_store<GROUP>(v, r, qrow + (ok ? b : 0) * 64, ok, scale_needs_clamp(s16));
+                __half *sdst = reinterpret_cast<__half *>(scales) + row * nb + b;
+                if (ok && QUAROT_IN_RANGE(sdst, 2, scales, M * nb * 2))
+                    *sdst = s16;
+                uint8_t *qdst = qrow + (ok ? b : 0) * 64;
+                quant_pack_store<GROUP>(v, r, qdst, ok && QUAROT_IN_RANGE(qdst, 64, q, M * (K / 2)),
+                                        scale_needs_clamp(s16));
             }
         } else {
             // one scale per row: reduce the row maximum over the row's threads
@@ -525,9 +535,10 @@ block128_quant_kernel(const uint4 *__restrict__ x,     // [M, K] fp16, 8 per uin
             amax = active ? __uint_as_float(rowmax[rl]) : 0.f;
             __syncthreads();
             const float r = amax > 0.f ? kQmax / amax : 0.f;
-            if (row_ok && b0 == 0)
+            if (row_ok && b0 == 0 && QUAROT_IN_RANGE(reinterpret_cast<float *>(scales) + row, 4, scales, M * 4))
                 reinterpret_cast<float *>(scales)[row] = amax * scale_mul;
             auto store = [&](uint8_t *dst, bool ok) {
+                ok = ok && QUAROT_IN_RANGE(dst, kCodeBytes, q, M * (int64_t)K * kCodeBytes / 128);
                 if (BITS != 4)
                     quant_store_i8(v, r, reinterpret_cast<int8_t *>(dst), ok);
                 else

@@ -335,20 +335,22 @@ had_tc_quant_kernel(const __grid_constant__ CUtensorMap tmap,   // x as fp16 [M 
                         amax = fmaxf(amax, red[(set * 2 + c) * 4 + (wq ^ 1)]);
                     }
                     r = amax > 0.f ? kQmax / amax : 0.f;
-                    if (valid && ap == 0)
+                    if (valid && ap == 0 && QUAROT_IN_RANGE(reinterpret_cast<float *>(scales) + t, 4, scales, M * 4))
                         reinterpret_cast<float *>(scales)[t] = amax * scale_mul;
                 } else {
                     __half s16;
                     r = group_scale(amax, scale_mul, sqrt_n, s16);
                     clamp = scale_needs_clamp(s16);
-                    if (valid)
-                        reinterpret_cast<__half *>(scales)[t * m + ap] = s16;
+                    __half *sdst = reinterpret_cast<__half *>(scales) + t * m + ap;
+                    if (valid && QUAROT_IN_RANGE(sdst, 2, scales, M * m * 2))
+                        *sdst = s16;
                 }
                 uint8_t *dst = q + (valid ? t : 0) * ((int64_t)K * kCodeBytes / 128) + ap * kCodeBytes;
+                const bool st_ok = valid && QUAROT_IN_RANGE(dst, kCodeBytes, q, M * ((int64_t)K * kCodeBytes / 128));
                 if (BITS == 4)
-                    quant_pack_store<GROUP>(v, r, dst, valid, clamp);
+                    quant_pack_store<GROUP>(v, r, dst, st_ok, clamp);
                 else
-                    quant_store_i8(v, r, reinterpret_cast<int8_t *>(dst), valid);
+                    quant_store_i8(v, r, reinterpret_cast<int8_t *>(dst), st_ok);
             }
         }
     }

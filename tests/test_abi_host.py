@@ -188,3 +188,13 @@ def test_fused_decode_rejects(q):
     assert f(A16, 64, A16, A16, None, A16, A16, 1, 16, 8, 128, A16, None) == 1
     assert f(A16, 64, A16, A16, A16, MIS, A16, 1, 16, 8, 128, A16, None) == 3
     assert f(None, 64, None, None, None, None, None, 0, 16, 8, 128, None, None) == 0   # empty batch
+
+
+def test_bounds_checking_build(q):
+    # the twin library compiled with QUAROT_DEBUG_BOUNDS says so; the normal one does not
+    from rotation_bit_quantization_randomized_b200 import build_lib
+    dbg = ctypes.CDLL(build_lib.LIB_DEBUG)
+    dbg.quarot_debug_bounds.restype = ctypes.c_int
+    assert dbg.quarot_debug_bounds() == 1
+    assert q.lib.quarot_debug_bounds() == (1 if q.DEBUG_BOUNDS else 0)
+    assert q.status_string(7) == "QUAROT_ERR_DEVICE_BOUNDS"
