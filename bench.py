@@ -71,7 +71,10 @@ KERNEL_SOURCES = {
     "had_tc_quant_kernel": ["rotate_tc.cuh", "rotate_quant.cuh", "kron_quant.cuh", "int4_gemm.cuh", "tc_ptx.cuh",
                             "common.cuh"],
     "kv_quant_tma_kernel_keys": ["kv_quant.cuh", "rotate_quant.cuh", "tc_ptx.cuh", "common.cuh"],
-    "kv_scores_kernel": ["kv_scores.cuh", "common.cuh"],
+    "kv_scores_tc_kernel": ["kv_scores_tc.cuh", "kv_decode_tc.cuh", "kron_quant.cuh", "int4_gemm.cuh",
+                            "rotate_quant.cuh", "kv_attend.cuh", "tc_ptx.cuh", "common.cuh"],
+    "kv_decode_tc_kernel": ["kv_decode_tc.cuh", "kron_quant.cuh", "int4_gemm.cuh", "rotate_quant.cuh",
+                            "kv_attend.cuh", "tc_ptx.cuh", "common.cuh"],
     "kv_attend_kernel": ["kv_attend.cuh", "common.cuh"],
     "kron_quant_kernel": ["kron_quant.cuh", "int4_gemm.cuh", "rotate_quant.cuh", "tc_ptx.cuh", "common.cuh"],
 }

@@ -252,6 +252,73 @@ __device__ __forceinline__ float dec_pow2_scale(float amax, float &inv)
     return __uint_as_float((uint32_t)(127 + e) << 23);
 }
 
+// The G queries of one KV head rotated and written as the B operand of the
+// score MMAs (threads 0-127; 16 threads per query, 8 elements each: bits 0-2
+// of the element index in registers, bits 3-6 through half-warp shuffles):
+//   q'[g] = (q[g] * diag(s_h)) H_128 / sqrt(128)  in fp32,
+// then per query the power of two 2^e of dec_pow2_scale and its hi / lo fp16
+// rows (dec_put_split) in the converted dim order; inv_qs[g] = 2^-e.
+// qg: the G query rows [G][128] fp16; sg: the head's 128 signs.
+template <int G>
+__device__ __forceinline__ void dec_rotate_queries(const __half *__restrict__ qg, const int8_t *__restrict__ sgn,
+                                                   uint8_t *bq, float *inv_qs, int tid)
+{
+    const float kInvSqrtD = 0.08838834764831845f;
+    const int p = tid & 15;
+    const int8_t *sg = sgn + 8 * p;
+#pragma unroll
+    for (int g0 = 0; g0 < G; g0 += kDecCompute / 16) {
+        const int g = g0 + (tid >> 4);
+        const bool gv = G % (kDecCompute / 16) == 0 || g < G;
+        const uint4 raw = gv ? *reinterpret_cast<const uint4 *>(qg + (int64_t)g * 128 + 8 * p)
+                             : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+        float v[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 f = half2_bits_to_float2(w4[k]);
+            v[2 * k] = sg[2 * k] < 0 ? -f.x : f.x;
+            v[2 * k + 1] = sg[2 * k + 1] < 0 ? -f.y : f.y;
+        }
+#pragma unroll
+        for (int hb = 1; hb < 8; hb <<= 1)
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if ((i & hb) == 0) {
+                    const float a = v[i], c = v[i + hb];
+                    v[i] = a + c;
+                    v[i + hb] = a - c;
+                }
+#pragma unroll
+        for (int lb = 1; lb < 16; lb <<= 1) {
+            const bool upper = (p & lb) != 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float o = __shfl_xor_sync(0xffffffffu, v[i], lb);
+                v[i] = upper ? o - v[i] : v[i] + o;
+            }
+        }
+        float mx = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            v[i] *= kInvSqrtD;
+            mx = fmaxf(mx, fabsf(v[i]));
+        }
+#pragma unroll
+        for (int lb = 1; lb < 16; lb <<= 1)
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, lb));
+        float inv;
+        const float sc = dec_pow2_scale(mx, inv);
+        if (gv) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                dec_put_split<G>(bq, g, 8 * p + dec_dim(i), v[i] * sc);
+            if (p == 0)
+                inv_qs[g] = inv;
+        }
+    }
+}
+
 template <int G>
 __global__ void __launch_bounds__(kDecThreads, G <= 8 ? 3 : 2)
 kv_decode_tc_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
@@ -289,7 +356,6 @@ kv_decode_tc_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
     const int Hq = Hkv * G;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool compute = warp < kDecCompute / 32;
-    const float kInvSqrtD = 0.08838834764831845f;
     // softmax in base 2: scores / sqrt(128) times log2(e), then exp2
     const float kScoreMul = 0.08838834764831845f * 1.4426950408889634f;
     const int64_t slice = (T + nsplit - 1) / nsplit;
@@ -342,65 +408,7 @@ kv_decode_tc_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
         vm = warp_max(vm, 32);
         if (lane == 0)
             vmx[warp] = vm;
-        // ---- rotate the G queries (16 threads per query, 8 elements each: bits
-        // 0-2 in registers, bits 3-6 through half-warp shuffles), as in the
-        // decode-scores kernel; the 16 threads of a query then find its maximum
-        // and write its hi / lo rows of B_q in the converted dim order
-        {
-            const int p = tid & 15;
-            const int8_t *sg = signs + h * 128 + 8 * p;
-    #pragma unroll
-            for (int g0 = 0; g0 < G; g0 += kDecCompute / 16) {
-                const int g = g0 + (tid >> 4);
-                const bool gv = G % (kDecCompute / 16) == 0 || g < G;
-                const uint4 raw = gv ? *reinterpret_cast<const uint4 *>(q + (b * Hq + (int64_t)h * G + g) * 128 + 8 * p)
-                                     : make_uint4(0u, 0u, 0u, 0u);
-                const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-                float v[8];
-    #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float2 f = half2_bits_to_float2(w4[k]);
-                    v[2 * k] = sg[2 * k] < 0 ? -f.x : f.x;
-                    v[2 * k + 1] = sg[2 * k + 1] < 0 ? -f.y : f.y;
-                }
-    #pragma unroll
-                for (int hb = 1; hb < 8; hb <<= 1)
-    #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        if ((i & hb) == 0) {
-                            const float a = v[i], c = v[i + hb];
-                            v[i] = a + c;
-                            v[i + hb] = a - c;
-                        }
-    #pragma unroll
-                for (int lb = 1; lb < 16; lb <<= 1) {
-                    const bool upper = (p & lb) != 0;
-    #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float o = __shfl_xor_sync(0xffffffffu, v[i], lb);
-                        v[i] = upper ? o - v[i] : v[i] + o;
-                    }
-                }
-                float mx = 0.f;
-    #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    v[i] *= kInvSqrtD;
-                    mx = fmaxf(mx, fabsf(v[i]));
-                }
-    #pragma unroll
-                for (int lb = 1; lb < 16; lb <<= 1)
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, lb));
-                float inv;
-                const float sc = dec_pow2_scale(mx, inv);
-                if (gv) {
-    #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        dec_put_split<G>(bq, g, 8 * p + dec_dim(i), v[i] * sc);
-                    if (p == 0)
-                        inv_qs[g] = inv;
-                }
-            }
-        }
+        dec_rotate_queries<G>(q + (b * Hq + (int64_t)h * G) * 128, signs + h * 128, bq, inv_qs, tid);
     }
     fence_proxy_async_smem();
     tc_fence_before();

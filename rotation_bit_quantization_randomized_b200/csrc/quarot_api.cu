@@ -1,6 +1,6 @@
 // quarot_api.cu -- the C ABI of libquarot (declared in include/quarot.h):
 // argument validation, launch configuration and error reporting around the
-// kernels in rotate_quant.cuh, int4_gemm.cuh and kv_scores.cuh.
+// kernels of the csrc/*.cuh headers.
 #include "quarot.h"
 
 #include "common.cuh"
@@ -10,8 +10,8 @@
 #include "kron_quant.cuh"
 #include "kv_attend.cuh"
 #include "kv_decode_tc.cuh"
+#include "kv_scores_tc.cuh"
 #include "kv_quant.cuh"
-#include "kv_scores.cuh"
 #include "mma_peak.cuh"
 #include "rotate_quant.cuh"
 #include "rotate_tc.cuh"
@@ -807,63 +807,125 @@ quarot_status_t attend_resident_clusters(int G, int split, int dev, int &fit)
     return QUAROT_OK;
 }
 
+// CTAs of a tensor-core decode kernel (the fused step or the scores) that can
+// be resident on one SM, computed from the kernel's own resources: shared
+// memory with the per-CTA reservation, registers in 256-register warp
+// allocations, threads, CTA slots.  The runtime's occupancy queries report
+// one CTA per SM for these kernels at any shared-memory size, while three are
+// resident when they run (counted on B200 with %smid).  Also raises the
+// kernel's dynamic shared-memory limit and asks for all of the unified L1 /
+// shared storage as shared memory.
+template <typename K>
+quarot_status_t tc_decode_per_sm(K kernel, size_t smem, int dev, int &per_sm)
+{
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaFuncSetAttribute");
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaFuncSetAttribute");
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, kernel);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaFuncGetAttributes");
+    int smem_sm = 0, smem_res = 0, regs_sm = 0, thr_sm = 0, blk_sm = 0;
+    if (cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&smem_res, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&thr_sm, cudaDevAttrMaxThreadsPerMultiProcessor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&blk_sm, cudaDevAttrMaxBlocksPerMultiprocessor, dev) != cudaSuccess)
+        return fail(QUAROT_ERR_CUDA, "cudaDeviceGetAttribute failed");
+    const int warp_regs = ((fa.numRegs * 32 + 255) / 256) * 256;
+    const int cta_regs = warp_regs * (kDecThreads / 32);
+    const int cta_smem = (int)smem + (int)fa.sharedSizeBytes + smem_res;
+    per_sm = std::min(std::min(smem_sm / cta_smem, regs_sm / std::max(cta_regs, 1)),
+                      std::min(thr_sm / kDecThreads, blk_sm));
+    if (per_sm < 1)
+        return fail(QUAROT_ERR_CUDA, "a decode kernel does not fit on an SM");
+    return QUAROT_OK;
+}
+
 // Clusters of `split` fused decode CTAs (G query heads per KV head) that can
-// be resident at once, computed once per (device, G); also raises the
-// kernel's dynamic shared-memory limit.  The count comes from the kernel's
-// own resources (shared memory with the per-CTA reservation, registers in
-// 256-register warp allocations, threads, CTA slots): the runtime's occupancy
-// queries report one CTA per SM for this kernel at any shared-memory size,
-// while up to three are resident when it runs (counted on B200 with %smid).
+// be resident at once (tc_decode_per_sm, computed once per (device, G)).
 template <int G>
 quarot_status_t decode_resident_clusters(int split, int dev, int &fit)
 {
     static int cache[kMaxDevices];
     static bool known[kMaxDevices];
-    int per_sm = 0, sms = 0;
+    int per_sm = 0;
     {
         std::lock_guard<std::mutex> lk(g_mutex);
         if (known[dev])
             per_sm = cache[dev];
     }
-    cudaError_t e;
     if (per_sm == 0) {
-        e = cudaFuncSetAttribute(kv_decode_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)DecShape<G>::kBytes);
-        if (e != cudaSuccess)
-            return cuda_fail(e, "cudaFuncSetAttribute");
-        // all of the unified L1 / shared storage as shared memory, so that
-        // several CTAs (about 75 KB each) share an SM
-        e = cudaFuncSetAttribute(kv_decode_tc_kernel<G>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 (int)cudaSharedmemCarveoutMaxShared);
-        if (e != cudaSuccess)
-            return cuda_fail(e, "cudaFuncSetAttribute");
-        cudaFuncAttributes fa;
-        e = cudaFuncGetAttributes(&fa, kv_decode_tc_kernel<G>);
-        if (e != cudaSuccess)
-            return cuda_fail(e, "cudaFuncGetAttributes");
-        int smem_sm = 0, smem_res = 0, regs_sm = 0, thr_sm = 0, blk_sm = 0;
-        if (cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&smem_res, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&thr_sm, cudaDevAttrMaxThreadsPerMultiProcessor, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&blk_sm, cudaDevAttrMaxBlocksPerMultiprocessor, dev) != cudaSuccess)
-            return fail(QUAROT_ERR_CUDA, "cudaDeviceGetAttribute failed");
-        const int warp_regs = ((fa.numRegs * 32 + 255) / 256) * 256;
-        const int cta_regs = warp_regs * (kDecThreads / 32);
-        const int cta_smem = (int)DecShape<G>::kBytes + (int)fa.sharedSizeBytes + smem_res;
-        per_sm = std::min(std::min(smem_sm / cta_smem, regs_sm / std::max(cta_regs, 1)),
-                          std::min(thr_sm / kDecThreads, blk_sm));
-        if (per_sm < 1)
-            return fail(QUAROT_ERR_CUDA, "kv_decode_tc_kernel does not fit on an SM");
+        quarot_status_t s = tc_decode_per_sm(kv_decode_tc_kernel<G>, DecShape<G>::kBytes, dev, per_sm);
+        if (s != QUAROT_OK)
+            return s;
         std::lock_guard<std::mutex> lk(g_mutex);
         cache[dev] = per_sm;
         known[dev] = true;
     }
-    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int sms = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess)
         return cuda_fail(e, "cudaDeviceGetAttribute");
     fit = sms * per_sm / split;
     return QUAROT_OK;
+}
+
+// The scores on the tensor cores: CTAs of `tiles_per_cta` consecutive
+// 128-token tiles of one (batch, KV head).  A CTA costs about its tiles plus
+// half a tile of set-up (query rotation, tensor-memory allocation); the
+// launch about ceil(CTAs / resident CTAs) such costs.  The tile count with the
+// smallest estimate.
+template <int G>
+quarot_status_t launch_scores_tc(const __half *q, const int8_t *signs, const uint8_t *kq, const __half *ks,
+                                 int64_t B, int64_t T, int Hkv, float *scores, cudaStream_t st, int dev)
+{
+    static int cache[kMaxDevices];
+    static bool known[kMaxDevices];
+    int per_sm = 0;
+    {
+        std::lock_guard<std::mutex> lk(g_mutex);
+        if (known[dev])
+            per_sm = cache[dev];
+    }
+    if (per_sm == 0) {
+        quarot_status_t s = tc_decode_per_sm(kv_scores_tc_kernel<G>, ScShape<G>::kBytes, dev, per_sm);
+        if (s != QUAROT_OK)
+            return s;
+        std::lock_guard<std::mutex> lk(g_mutex);
+        cache[dev] = per_sm;
+        known[dev] = true;
+    }
+    int sms = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaDeviceGetAttribute");
+    const int64_t slots = (int64_t)sms * per_sm;
+    const int64_t tiles = (T + kDecTile - 1) / kDecTile;
+    int64_t best_tpc = 1;
+    double best = -1.0;
+    for (int64_t tpc = 1;; tpc *= 2) {
+        const int64_t chunks = (tiles + tpc - 1) / tpc;
+        const int64_t ctas = B * Hkv * chunks;
+        const double est = (double)((ctas + slots - 1) / slots) * ((double)std::min(tpc, tiles) + 0.5);
+        if (chunks <= 0x7fffffff && (best < 0.0 || est < best)) {
+            best = est;
+            best_tpc = tpc;
+        }
+        if (tpc >= tiles)
+            break;
+    }
+    const int64_t chunks = (tiles + best_tpc - 1) / best_tpc;
+    if (chunks > 0x7fffffff)
+        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "T too large");
+    dim3 grid((unsigned)chunks, (unsigned)Hkv, (unsigned)B);
+    kv_scores_tc_kernel<G><<<grid, kDecThreads, ScShape<G>::kBytes, st>>>(q, signs, kq, ks, T, Hkv, (int)best_tpc,
+                                                                          scores);
+    return after_launch("kv_scores_tc_kernel launch");
 }
 
 template <int G>
@@ -1331,22 +1393,17 @@ quarot_status_t quarot_kv_decode_scores(const void *q_f16, int64_t Hq, const int
     quarot_status_t s = current_device(dev, info);
     if (s != QUAROT_OK)
         return s;
-    const int64_t chunks = (T + kScoreTokPerCta - 1) / kScoreTokPerCta;
-    if (chunks > 0x7fffffff)
-        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "T too large");
-    dim3 grid((unsigned)chunks, (unsigned)Hkv, (unsigned)B);
     cudaStream_t st = (cudaStream_t)stream;
     const __half *qh = static_cast<const __half *>(q_f16);
-    const uint4 *k4 = reinterpret_cast<const uint4 *>(kq);
     const __half *ksh = static_cast<const __half *>(ks_f16);
+    const int hkv = (int)Hkv;
     switch (G) {
-    case 1: kv_scores_kernel<1><<<grid, kScoreThreads, 0, st>>>(qh, signs, k4, ksh, T, (int)Hkv, scores); break;
-    case 2: kv_scores_kernel<2><<<grid, kScoreThreads, 0, st>>>(qh, signs, k4, ksh, T, (int)Hkv, scores); break;
-    case 4: kv_scores_kernel<4><<<grid, kScoreThreads, 0, st>>>(qh, signs, k4, ksh, T, (int)Hkv, scores); break;
-    case 8: kv_scores_kernel<8><<<grid, kScoreThreads, 0, st>>>(qh, signs, k4, ksh, T, (int)Hkv, scores); break;
-    default: kv_scores_kernel<16><<<grid, kScoreThreads, 0, st>>>(qh, signs, k4, ksh, T, (int)Hkv, scores); break;
+    case 1: return launch_scores_tc<1>(qh, signs, kq, ksh, B, T, hkv, scores, st, dev);
+    case 2: return launch_scores_tc<2>(qh, signs, kq, ksh, B, T, hkv, scores, st, dev);
+    case 4: return launch_scores_tc<4>(qh, signs, kq, ksh, B, T, hkv, scores, st, dev);
+    case 8: return launch_scores_tc<8>(qh, signs, kq, ksh, B, T, hkv, scores, st, dev);
+    default: return launch_scores_tc<16>(qh, signs, kq, ksh, B, T, hkv, scores, st, dev);
     }
-    return after_launch("kv_scores_kernel launch");
 }
 
 quarot_status_t quarot_kv_decode_attend(const float *scores, int64_t B, int64_t Hq, const uint8_t *vq,

@@ -150,3 +150,21 @@ def test_decode_full_size_sampled_batches(q):
     bound = _bound(qh[rows], s, kq_n, ks_n, vq_n, vs_n)
     err = np.abs(got.cpu().numpy()[rows].astype(np.float64) - ref)
     assert np.all(err <= bound), f"max error / bound {np.max(err / bound):.3f}"
+
+
+@pytest.mark.parametrize("B,T", [(1, 2048), (16, 2048), (2, 1000)])
+def test_decode_back_to_back(q, B, T):
+    # many launches on one stream with no synchronization between them: the
+    # same bytes as a lone launch, and no bounded wait runs out
+    rng = np.random.default_rng(B + T)
+    H, G = 8, 8
+    s, kq, ks, vq, vs = _cache(rng, B, T, H)
+    qh = rng.standard_normal((B, H * G, 128)).astype(np.float16)
+    args = (_dev(qh), _dev(s), _dev(kq), _dev(ks.view(np.float16)), _dev(vq), _dev(vs.view(np.float16)))
+    ref = q.quarot_kv_decode_attention(*args)
+    _ok(q)
+    out = torch.empty_like(ref)
+    for _ in range(60):
+        q.quarot_kv_decode_attention(*args, out)
+    _ok(q)
+    assert torch.equal(out, ref)

@@ -109,3 +109,25 @@ def test_kv_scores_full_size_sampled(q):
     k, v, qh, s = synth.kv_inputs(c, batch=4)
     kq, ks, _, _ = oracle.kv_quant(k, v, s)
     _scores_check(q, qh, s, kq, ks)
+
+
+@pytest.mark.parametrize("B,T", [(1, 2048), (4, 2048), (2, 1000), (3, 129)])
+def test_kv_scores_back_to_back(q, B, T):
+    # many launches on one stream with no synchronization between them: every
+    # one gives the same bytes as a lone launch and no wait runs out (a
+    # hand-off barrier that could run two phases ahead of its waiter would
+    # show here as a timeout)
+    rng = np.random.default_rng(B * T)
+    H, G = 8, 8
+    k = rng.standard_normal((B, T, H, 128)).astype(np.float16)
+    s = np.stack([synth.signs(128, 40 + h) for h in range(H)])
+    kq, ks, _, _ = oracle.kv_quant(k, np.zeros_like(k), s)
+    qh = rng.standard_normal((B, H * G, 128)).astype(np.float16)
+    args = (_dev(qh), _dev(s), _dev(kq), _dev(ks.view(np.float16)))
+    ref = q.quarot_kv_decode_scores(*args)
+    _ok(q)
+    out = torch.empty_like(ref)
+    for _ in range(60):
+        q.quarot_kv_decode_scores(*args, out)
+    _ok(q)
+    assert torch.equal(out, ref)
