@@ -14,8 +14,12 @@
 // The tiles use the 128-byte swizzle (two boxes of 64 columns), so that the
 // 16-byte chunk c of row r sits at chunk c ^ (r mod 8) of its 128-byte line
 // and the row-per-thread reads of a warp hit every bank evenly.
-// Requires Hkv to divide 128: then every row a thread handles belongs to the
-// same KV head, and its sign words are built once.
+// When Hkv divides 128, every row a thread handles belongs to the same KV
+// head, and its sign words are built once; otherwise the CTA builds every
+// head's sign words into a table in shared memory once, and each thread
+// reads its row's entry per tile.  (The block rotation I_{K/128} (x) H_128
+// with 128-groups is the same computation on the rows of x viewed as
+// [M K/128, 128], with K/128 "heads" of 128 signs.)
 #pragma once
 
 #include <cuda.h>
@@ -28,7 +32,9 @@ namespace quarot {
 constexpr int kKvTileRows = 128;
 constexpr int kKvStages = 3;
 constexpr int kKvStageBytes = kKvTileRows * 256;          // two 64-column boxes of 16 KB
-constexpr int kKvSmemBytes = kKvStages * kKvStageBytes + 64 + 1024;
+constexpr int kKvMaxHeads = 512;                         // sign-word table: 16 bytes per head
+constexpr int kKvSgnOffset = kKvStages * kKvStageBytes + 64;
+constexpr int kKvSmemBytes = kKvSgnOffset + kKvMaxHeads * 16 + 1024;
 constexpr uint64_t kKvWaitLimitNs = 2000000000ull;
 
 template <bool ROTATE>
@@ -56,6 +62,16 @@ kv_quant_tma_kernel(const __grid_constant__ CUtensorMap tmap,   // fp16 [rows, 1
         mbar_fence_init();
         tma_prefetch_desc(&tmap);
     }
+    // heads that change from tile to tile (hkv does not divide 128): every
+    // head's sign words, built once per CTA
+    const bool head_per_tile = ROTATE && (kKvTileRows % hkv) != 0;
+    uint4 *sgn_tab = reinterpret_cast<uint4 *>(smem + kKvSgnOffset);
+    if (head_per_tile)
+        for (int hh = t; hh < hkv; hh += kKvTileRows) {
+            uint32_t w4[4];
+            build_sign_words(signs + (int64_t)hh * 128, [&](int j) { return 2 * j; }, w4);
+            sgn_tab[hh] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
     __syncthreads();
 
     int issued = 0;                       // thread 0: tiles whose copies were issued (in tile order)
@@ -74,9 +90,9 @@ kv_quant_tma_kernel(const __grid_constant__ CUtensorMap tmap,   // fp16 [rows, 1
                 issue(first + s * step, s);
     }
 
-    // sign words of this thread's head (the same for every tile: hkv divides 128)
+    // sign words of this thread's head (the same for every tile when hkv divides 128)
     uint32_t sgn[4] = {0u, 0u, 0u, 0u};
-    if (ROTATE) {
+    if (ROTATE && !head_per_tile) {
         const int8_t *sh = signs + (int64_t)(t % hkv) * 128;
         build_sign_words(sh, [&](int j) { return 2 * j; }, sgn);
     }
@@ -111,6 +127,13 @@ kv_quant_tma_kernel(const __grid_constant__ CUtensorMap tmap,   // fp16 [rows, 1
             for (int c = 0; c < 8; ++c)
                 w[8 * h + c] = *reinterpret_cast<const uint4 *>(base + h * (kKvStageBytes / 2) + ((c ^ (t & 7)) << 4));
         __syncthreads();                  // every read of stage s is done: it may be refilled
+        if (head_per_tile) {
+            const uint4 w4 = sgn_tab[(tile * kKvTileRows + t) % hkv];
+            sgn[0] = w4.x;
+            sgn[1] = w4.y;
+            sgn[2] = w4.z;
+            sgn[3] = w4.w;
+        }
         float v[128];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {

@@ -26,6 +26,12 @@
 
 using namespace quarot;
 
+// The staged KV-write launcher (defined below, outside the internal namespace).
+template <bool ROTATE>
+quarot_status_t launch_kv_tma(const void *x, int64_t rows, int hkv, const int8_t *signs, uint8_t *q, void *scales,
+                              float scale_mul, float sqrt_n, cudaStream_t st, int dev, int sms,
+                              uint64_t wait_limit_ns = kKvWaitLimitNs, int64_t withheld_tile = -1);
+
 namespace {
 
 thread_local std::string g_last_error;
@@ -319,6 +325,11 @@ quarot_status_t rotate_quant_launch(const void *x, int64_t M, int64_t K, const i
     }
     const float mul = (float)(1.0 / (qmax_of(bits) * std::sqrt(128.0)));
     const float sq = (float)std::sqrt(128.0);
+    const int64_t nb = K / 128;
+    if (bits == 4 && group == 128 && nb <= kKvMaxHeads && M * nb < (int64_t(1) << 31) - kKvTileRows)
+        // I_{K/128} (x) H_128 with 128-groups: the KV write's computation on x
+        // viewed as [M K/128, 128] rows, head = block index
+        return launch_kv_tma<true>(x, M * nb, (int)nb, signs, q, scales, mul, sq, st, dev, sms);
     if (bits == 8)
         return launch_block<true, 0, 8>(x, M, K, signs, q, scales, mul, sq, st, dev, sms);
     if (bits == 6)
@@ -997,11 +1008,11 @@ quarot_status_t kv_map(CUtensorMap &map, const void *base, int64_t rows)
     return QUAROT_OK;
 }
 
-// The staged KV-write kernel over `rows` rows of 128 elements (Hkv divides 128).
+// The staged KV-write kernel over `rows` rows of 128 elements, row r of head r mod hkv.
 template <bool ROTATE>
 quarot_status_t launch_kv_tma(const void *x, int64_t rows, int hkv, const int8_t *signs, uint8_t *q, void *scales,
                               float scale_mul, float sqrt_n, cudaStream_t st, int dev, int sms,
-                              uint64_t wait_limit_ns = kKvWaitLimitNs, int64_t withheld_tile = -1)
+                              uint64_t wait_limit_ns, int64_t withheld_tile)
 {
     auto kern = kv_quant_tma_kernel<ROTATE>;
     int per_sm = 0;
@@ -1351,8 +1362,8 @@ quarot_status_t quarot_kv_quant(const void *k_f16, const void *v_f16, int64_t B,
     cudaStream_t st = (cudaStream_t)stream;
     const float kmul = (float)(1.0 / (7.0 * std::sqrt(128.0)));
     const float ksq = (float)std::sqrt(128.0);
-    if (128 % Hkv == 0 && rows * Hkv < (int64_t(1) << 31) - kKvTileRows) {
-        // rows of one head staged by the copy engine; every thread keeps one head
+    if (rows * Hkv < (int64_t(1) << 31) - kKvTileRows) {
+        // rows of [B T Hkv, 128] staged by the copy engine
         const int64_t n = rows * Hkv;
         s = launch_kv_tma<true>(k_f16, n, (int)Hkv, signs, kq, ks_f16, kmul, ksq, st, dev, info->sm_count);
         if (s != QUAROT_OK)
