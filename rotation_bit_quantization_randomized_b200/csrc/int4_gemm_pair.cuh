@@ -43,6 +43,16 @@
 //    leaves while its peer may still read its memory or signal it.
 // All waits are bounded in time, as in the single-CTA kernel; waits in front
 // of warp-collective tcgen05 instructions are warp-uniform.
+//
+// Grouped scales (EPI == kEpiGroupF16, 128-wide K groups, N tile 128 per
+// pair): every K step is its own int32 accumulation, into one of three
+// 128-column accumulators that rotate step by step (four A stages fill the
+// rest of tensor memory); eight epilogue warps per CTA (two per lane
+// quarter, 64 columns each) read each step's partial sums, convert them
+// exactly, scale them by the step's row and column scales (staged in shared
+// memory eight groups at a time) and accumulate in fp32 registers; the MMA
+// thread waits for an accumulator's previous partial sums to be read before
+// it starts the next step in it.
 #pragma once
 
 #include "int4_gemm.cuh"
@@ -53,6 +63,7 @@ constexpr int kPairBM = 256;       // output rows per CTA pair
 
 template <int BN, int EPI>
 struct PairShape {
+    static constexpr bool kGrouped = EPI == kEpiGroupF16;
     static constexpr int kRowsA = kPairBM / 2;                        // A rows per CTA
     static constexpr int kRowsB = BN / 2;                             // B rows per CTA
     static constexpr int kPackedA = kRowsA * kGemmBK / 2;             // 8 KB, 64-byte swizzled
@@ -60,25 +71,35 @@ struct PairShape {
     static constexpr int kPackedStage = kPackedA + kPackedB;
     static constexpr int kBBytes = kRowsB * kGemmBK;                  // widened B stage
     static constexpr int kTmemCols = 512;
-    static constexpr int kAStages = (kTmemCols - 2 * BN) / 32;       // int8 A stages in tensor memory
+    static constexpr int kAccBufs = kGrouped ? 3 : 2;                // accumulators of BN columns
+    static constexpr int kAStages = (kTmemCols - kAccBufs * BN) / 32; // int8 A stages in tensor memory
     static constexpr int kBStages = 4;                                // int8 B stages in shared memory
     static constexpr int kPStages = 8;
     static constexpr int kBGroups = kRowsB / 8;                       // groups of 8 B rows
     static constexpr int kUnpackWarps = 4;                            // per group: one per TMEM lane quarter
-    static constexpr int kUnpackGroups = 2;                           // groups take alternate K steps
+    // groups take alternate K steps; the grouped kernel keeps one, because its
+    // eight epilogue warps hold 64 fp32 sums each and 18 warps would leave
+    // them too few registers (measured: 2.40 ms with one group against 2.79
+    // ms with two, which spill, at 4096 x 28672 x 8192)
+    static constexpr int kUnpackGroups = kGrouped ? 1 : 2;
     static constexpr int kBGroupsPerWarp = (kBGroups + kUnpackWarps - 1) / kUnpackWarps;
     static constexpr int kUnpackArrivals = kUnpackWarps;              // one arrival per warp and stage
-    static constexpr int kEpiWarps = 4;
-    static constexpr int kMmaWarp = 4;
-    static constexpr int kTmaWarp = 5;
-    static constexpr int kUnpackWarp0 = 6;
+    static constexpr int kEpiWarps = kGrouped ? 8 : 4;
+    static constexpr int kEpiThreads = 32 * kEpiWarps;
+    static constexpr int kMmaWarp = kEpiWarps;
+    static constexpr int kTmaWarp = kEpiWarps + 1;
+    static constexpr int kUnpackWarp0 = kEpiWarps + 2;
     static constexpr int kThreads = 32 * (kUnpackWarp0 + kUnpackGroups * kUnpackWarps);
-    static constexpr int kACol0 = 2 * BN;                             // A stage s at kACol0 + 32 s
+    static constexpr int kACol0 = kAccBufs * BN;                      // A stage s at kACol0 + 32 s
     static constexpr int kIntOffset = kPStages * kPackedStage;
     static constexpr int kBarOffset = kIntOffset + kBStages * kBBytes;
-    static constexpr int kNumBars = 2 * kPStages + 2 * kBStages + 5;
+    static constexpr int kNumBars = 2 * kPStages + 2 * kBStages + 2 * kAccBufs + 1;
     static constexpr int kMiscOffset = kBarOffset + 8 * kNumBars;
-    static constexpr int kSmemBytes = kMiscOffset + 16 + 1024;
+    static constexpr int kGroupChunk = 8;                             // K groups per staged scale chunk
+    static constexpr int kSwOffset = kMiscOffset + 16;                // grouped: [2][8][128] row, [2][8][BN] column scales
+    static constexpr int kSmemBytes = kSwOffset + (kGrouped ? 2 * kGroupChunk * (kRowsA + BN) * 4 : 0) + 1024;
+    static_assert(!kGrouped || (BN == 128 && kEpiThreads == kRowsA + BN),
+                  "grouped: N tile 128, one scale-staging thread per tile row and column");
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
     static_assert(kPackedStage % 1024 == 0 && kBBytes % 1024 == 0, "1024-byte aligned stages");
     static_assert(kRowsB % 8 == 0 && BN % 32 == 0 && BN <= 256, "B rows in groups of 8; N tile of whole column chunks");
@@ -104,8 +125,8 @@ int4_gemm_pair_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_
     const uint32_t bar_ifull = bar_pempty + 8 * S::kPStages;       // used in the leader
     const uint32_t bar_sdone = bar_ifull + 8 * S::kBStages;        // MMAs of step s done (slot s % kBStages)
     const uint32_t bar_accf = bar_sdone + 8 * S::kBStages;
-    const uint32_t bar_acce = bar_accf + 16;                       // used in the leader
-    const uint32_t bar_drain = bar_acce + 16;
+    const uint32_t bar_acce = bar_accf + 8 * S::kAccBufs;          // used in the leader
+    const uint32_t bar_drain = bar_acce + 8 * S::kAccBufs;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + S::kMiscOffset);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + S::kMiscOffset + 4);
 
@@ -129,7 +150,7 @@ int4_gemm_pair_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_
             mbar_init(bar_ifull + 8 * s, 2 * S::kUnpackArrivals);   // leader's: both CTAs' unpackers
             mbar_init(bar_sdone + 8 * s, 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < S::kAccBufs; ++b) {
             mbar_init(bar_accf + 8 * b, 1);
             mbar_init(bar_acce + 8 * b, 2 * S::kEpiWarps);
         }
@@ -281,11 +302,21 @@ int4_gemm_pair_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_
             int step = 0;
             for (int lt = 0; lt < my_tiles && ok; ++lt) {
                 const int ab = lt & 1;
-                if (!gemm_wait(bar_acce + 8 * ab, ((uint32_t)(lt >> 1) & 1) ^ 1, abort_flag))
+                if (!S::kGrouped && !gemm_wait(bar_acce + 8 * ab, ((uint32_t)(lt >> 1) & 1) ^ 1, abort_flag))
                     break;
                 tc_fence_after();
-                const uint32_t d = tmem_base + ab * BN;
+                uint32_t d = tmem_base + ab * BN;
                 for (int kb = 0; kb < KB; ++kb, ++step) {
+                    if (S::kGrouped) {
+                        // step's own accumulator: free once the epilogue has read
+                        // the partial sums of step - kAccBufs
+                        const int gb = step % S::kAccBufs;
+                        if (!gemm_wait(bar_acce + 8 * gb, ((uint32_t)(step / S::kAccBufs) & 1) ^ 1, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        d = tmem_base + gb * BN;
+                    }
                     const int bsi = step % S::kBStages;
                     if (!gemm_wait(bar_ifull + 8 * bsi, (uint32_t)(step / S::kBStages) & 1, abort_flag)) {
                         ok = false;
@@ -297,9 +328,11 @@ int4_gemm_pair_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
                         umma_i8_ts_pair(d, at + 8 * j, desc_kmajor_sw128(bs + 32 * j), idesc,
-                                        (kb > 0 || j > 0) ? 1u : 0u);
+                                        ((!S::kGrouped && kb > 0) || j > 0) ? 1u : 0u);
                     umma_commit_pair(bar_sdone + 8 * bsi, 0x3);
-                    if (kb == KB - 1)
+                    if (S::kGrouped)
+                        umma_commit_pair(bar_accf + 8 * (step % S::kAccBufs), 0x3);
+                    else if (kb == KB - 1)
                         umma_commit_pair(bar_accf + 8 * ab, 0x3);
                 }
             }
@@ -307,6 +340,138 @@ int4_gemm_pair_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tma_
             gemm_wait_drain(bar_drain, 0);
         }
         __syncwarp();
+    } else if constexpr (S::kGrouped) {
+        // ------------------------------------------------------------ grouped epilogue (both CTAs)
+        // Warps w and w + 4 share TMEM lane quarter w % 4 and split the 128
+        // columns.  The row and column scales of 8 K groups at a time are
+        // staged in shared memory one chunk ahead (threads 0-127: this CTA's
+        // 128 rows, 128-255: the tile's 128 columns); a named barrier of the
+        // epilogue warps hands each chunk over and makes every thread's
+        // decision to go on (or to give up after a timeout) the same.
+        constexpr int kCh = S::kGroupChunk;
+        constexpr int HALF = BN / 2;
+        const int wq = warp & 3;
+        const int col0 = (warp >> 2) * HALF;
+        const uint32_t lane_addr = tmem_base + ((uint32_t)(32 * wq) << 16);
+        const int et = threadIdx.x;                         // 0 .. kEpiThreads - 1
+        const int G = KB;
+        float *sac = reinterpret_cast<float *>(smem + S::kSwOffset);       // [2][kCh][kRowsA]
+        float *swc = sac + 2 * kCh * S::kRowsA;                            // [2][kCh][BN]
+        const bool is_row = et < S::kRowsA;
+        const float smul = is_row ? (1.0f / 256.0f) : 1.0f;                // both operands are 16 x code
+        bool ok = true;
+        int step = 0;
+        for (int lt = 0; lt < my_tiles && ok; ++lt) {
+            int mb, nb;
+            gemm_tile_coords(cluster + lt * nclusters, a.tiles_m, a.tiles_n, mb, nb);
+            const int64_t mrow0 = (int64_t)mb * kPairBM + S::kRowsA * rank;
+            const int64_t m = mrow0 + 32 * wq + lane;
+            const int64_t n0 = (int64_t)nb * BN;
+            const bool mrow = m < a.M;
+            const int64_t srow = is_row ? mrow0 + et : n0 + (et - S::kRowsA);
+            const bool sval = is_row ? srow < a.M : srow < a.N;
+            const __half *sptr = reinterpret_cast<const __half *>(is_row ? a.sa : a.sw) + (sval ? srow : 0) * G;
+            auto load_chunk = [&](int kb0, float (&d)[kCh]) {
+                if (sval && G % kCh == 0) {
+                    const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(sptr + kb0));
+                    const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float2 f = half2_bits_to_float2(w4[i]);
+                        d[2 * i] = f.x * smul;
+                        d[2 * i + 1] = f.y * smul;
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < kCh; ++i)
+                        d[i] = (sval && kb0 + i < G) ? __half2float(sptr[kb0 + i]) * smul : 0.f;
+                }
+            };
+            auto store_chunk = [&](int cb, const float (&d)[kCh]) {
+#pragma unroll
+                for (int i = 0; i < kCh; ++i) {
+                    if (is_row)
+                        sac[(cb * kCh + i) * S::kRowsA + et] = d[i];
+                    else
+                        swc[(cb * kCh + i) * BN + (et - S::kRowsA)] = d[i];
+                }
+            };
+            float accv[HALF];
+#pragma unroll
+            for (int i = 0; i < HALF; ++i)
+                accv[i] = 0.f;
+            {
+                float d[kCh];
+                load_chunk(0, d);
+                store_chunk(0, d);
+            }
+            for (int kb0 = 0; kb0 < KB; kb0 += kCh) {
+                const int cb = (kb0 / kCh) & 1;
+                ok = epi_barrier_and(S::kEpiThreads, ok);
+                if (!ok)
+                    break;
+                float nxt[kCh];
+                if (kb0 + kCh < KB)
+                    load_chunk(kb0 + kCh, nxt);
+                const int nu = min(kCh, KB - kb0);
+                for (int u = 0; u < nu; ++u, ++step) {
+                    const int gb = step % S::kAccBufs;
+                    if (!gemm_wait_warp(bar_accf + 8 * gb, (uint32_t)(step / S::kAccBufs) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const float sag = sac[(cb * kCh + u) * S::kRowsA + 32 * wq + lane];
+                    const float *sws = swc + (cb * kCh + u) * BN;
+#pragma unroll
+                    for (int c = 0; c < HALF / 16; ++c) {
+                        uint32_t r[16];
+                        __syncwarp();
+                        tmem_ld16(lane_addr + gb * BN + col0 + 16 * c, r);
+                        tmem_wait_ld16(r);
+                        if (c == HALF / 16 - 1) {
+                            // both CTAs' 8 warps arrive on the leader's barrier
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0)
+                                mbar_arrive_remote(mapa_shared(bar_acce + 8 * gb, 0));
+                        }
+                        // two partial sums at a time: exact int -> float with one
+                        // packed subtract (|acc| < 2^22), times the column scales,
+                        // then accumulated with the row scale by one packed FMA
+#pragma unroll
+                        for (int i = 0; i < 16; i += 2) {
+                            float f0, f1;
+                            sub_x2(__uint_as_float(r[i] + 0x4B400000u), __uint_as_float(r[i + 1] + 0x4B400000u),
+                                   12582912.0f, f0, f1);
+                            const float2 w = *reinterpret_cast<const float2 *>(sws + col0 + 16 * c + i);
+                            mul_x2(f0, f1, w.x, w.y, f0, f1);
+                            fma_x2_acc(f0, f1, sag, accv[16 * c + i], accv[16 * c + i + 1]);
+                        }
+                    }
+                }
+                if (kb0 + kCh < KB)
+                    store_chunk(cb ^ 1, nxt);
+            }
+            ok = epi_barrier_and(S::kEpiThreads, ok);
+            if (!ok)
+                break;
+            if (mrow) {
+                __half *orow = reinterpret_cast<__half *>(a.out) + m * a.N;
+#pragma unroll
+                for (int v = 0; v < HALF / 8; ++v) {
+                    const int64_t n = n0 + col0 + 8 * v;
+                    if (n < a.N) {
+                        uint32_t h[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            h[i] = h2_as_u32(__floats2half2_rn(accv[8 * v + 2 * i], accv[8 * v + 2 * i + 1]));
+                        if (QUAROT_IN_RANGE(orow + n, 16, a.out, a.M * a.N * 2))
+                            *reinterpret_cast<uint4 *>(orow + n) = make_uint4(h[0], h[1], h[2], h[3]);
+                    }
+                }
+            }
+        }
     } else {
         // ------------------------------------------------------------ epilogue (both CTAs)
         const int wq = warp & 3;

@@ -414,52 +414,6 @@ quarot_status_t packed_map(CUtensorMap &map, const uint8_t *base, int64_t rows, 
     return QUAROT_OK;
 }
 
-template <int BN, int EPI>
-quarot_status_t launch_gemm(GemmArgs a, cudaStream_t st, bool pdl)
-{
-    using S = GemmShape<BN, EPI>;
-    int dev;
-    DeviceInfo *info;
-    quarot_status_t s = current_device(dev, info);
-    if (s != QUAROT_OK)
-        return s;
-    auto kern = int4_gemm_kernel<BN, EPI>;
-    int per_sm = 0;
-    s = kernel_occupancy(kern, dev, S::kThreads, S::kSmemBytes, per_sm);
-    if (s != QUAROT_OK)
-        return s;
-    a.tiles_m = (int)((a.M + kGemmBM - 1) / kGemmBM);
-    a.tiles_n = (int)((a.N + BN - 1) / BN);
-    a.kblocks = (int)(a.K / kGemmBK);
-    const int64_t tiles = (int64_t)a.tiles_m * a.tiles_n;
-    if (tiles > 0x7fffffff)
-        return fail(QUAROT_ERR_UNSUPPORTED_SHAPE, "too many output tiles");
-    CUtensorMap map_a, map_b;
-    s = packed_map(map_a, a.qa, a.M, a.K, kGemmBM);
-    if (s != QUAROT_OK)
-        return s;
-    s = packed_map(map_b, a.qw, a.N, a.K, BN);
-    if (s != QUAROT_OK)
-        return s;
-    const int grid = (int)std::min<int64_t>(tiles, (int64_t)info->sm_count);
-
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(S::kThreads);
-    cfg.dynamicSmemBytes = S::kSmemBytes;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    if (pdl) {
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-    }
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a, map_a, map_b);
-    if (e != cudaSuccess)
-        return cuda_fail(e, "int4_gemm_kernel launch");
-    return after_launch("int4_gemm_kernel launch");
-}
 
 // N tile of the pair GEMM: two accumulator buffers of 224 columns leave
 // tensor memory for two A stages.
@@ -470,19 +424,21 @@ constexpr int kPairBN = 224;
 template <int EPI, bool UNS = false>
 quarot_status_t launch_gemm_pair(GemmArgs a, cudaStream_t st, bool pdl)
 {
-    using S = PairShape<kPairBN, EPI>;
+    // grouped scales: N tile 128 per pair (three accumulators in tensor memory)
+    constexpr int BN = EPI == kEpiGroupF16 ? 128 : kPairBN;
+    using S = PairShape<BN, EPI>;
     int dev;
     DeviceInfo *info;
     quarot_status_t s = current_device(dev, info);
     if (s != QUAROT_OK)
         return s;
-    auto kern = int4_gemm_pair_kernel<kPairBN, EPI, UNS>;
+    auto kern = int4_gemm_pair_kernel<BN, EPI, UNS>;
     int per_sm = 0;
     s = kernel_occupancy(kern, dev, S::kThreads, S::kSmemBytes, per_sm);
     if (s != QUAROT_OK)
         return s;
     a.tiles_m = (int)((a.M + kPairBM - 1) / kPairBM);
-    a.tiles_n = (int)((a.N + kPairBN - 1) / kPairBN);
+    a.tiles_n = (int)((a.N + BN - 1) / BN);
     a.kblocks = (int)(a.K / kGemmBK);
     const int64_t tiles = (int64_t)a.tiles_m * a.tiles_n;
     if (tiles > 0x7fffffff)
@@ -622,7 +578,7 @@ quarot_status_t linear_launch(const uint8_t *qa, const void *sa, int64_t M, cons
     a.M = M;
     a.N = N;
     a.K = K;
-    return group == 0 ? launch_gemm_pair<kEpiScaledF16>(a, st, pdl) : launch_gemm<128, kEpiGroupF16>(a, st, pdl);
+    return group == 0 ? launch_gemm_pair<kEpiScaledF16>(a, st, pdl) : launch_gemm_pair<kEpiGroupF16>(a, st, pdl);
 }
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
