@@ -408,10 +408,15 @@ quarot_status_t quarot_kv_quant(const void *k_f16, const void *v_f16, int64_t B,
  *   scores[b,hq,t] = sum_d q'[d] * kq[b,t,h,d] * ks[b,t,h]   (fp32; no 1/sqrt(D),
  *                no softmax)
  *
+ * The products run on the tensor cores and are exact: the codes as fp16, the
+ * fp32 query split into two fp16 parts that carry 22 of its bits; only the
+ * fp32 sums over d round.
+ *
  * q_f16   [B, Hq, D] fp16.   signs [Hkv, D] int8.
  * kq      [B, T, Hkv, D/2] packed codes, ks_f16 [B, T, Hkv] fp16 (from quarot_kv_quant).
  * scores  [B, Hq, T] fp32 output.
- * Limits: D == 128; Hq % Hkv == 0 with Hq / Hkv <= 16; B, T >= 0.
+ * Limits: D == 128; Hq / Hkv in {1, 2, 4, 8, 16}; B, Hkv <= 65535; B, T >= 0
+ * (B == 0 or T == 0 launches nothing).
  */
 quarot_status_t quarot_kv_decode_scores(const void *q_f16, int64_t Hq, const int8_t *signs,
                                         const uint8_t *kq, const void *ks_f16, int64_t B,
