@@ -195,6 +195,13 @@ __device__ __forceinline__ float dec_exp2(float x)
     return y;
 }
 
+// Brings the line holding p into L2 ahead of its load (no register, no
+// wait); only issued for addresses inside the caches.
+__device__ __forceinline__ void prefetch_l2(const void *p)
+{
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // Barrier of the four compute warps (named barrier 1, 128 threads); the MMA
 // warp never takes part.
 __device__ __forceinline__ void dec_bar_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
@@ -392,10 +399,23 @@ kv_decode_tc_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
                 w[c] = make_uint4(0u, 0u, 0u, 0u);
         }
     };
+    // token t of tile j, two tiles ahead of its register load: its code rows
+    // and scales into L2
+    auto prefetch_tile = [&](int j) {
+        const int64_t t = ts + (int64_t)j * kDecTile + tid;
+        if (j < ntiles && t < te) {
+            const int64_t r = (b * T + t) * Hkv + h;
+            prefetch_l2(kq + r * 64);
+            prefetch_l2(vq + r * 64);
+            prefetch_l2(ks + r);
+            prefetch_l2(vs + r);
+        }
+    };
     uint4 krow[4], vrow[4];
     if (compute) {
         load_row(kq, 0, krow);
         load_row(vq, 0, vrow);
+        prefetch_tile(1);
         // ---- the slice's largest value scale (the weights e * vs never
         // exceed it, so one power-of-two scale serves every tile of the slice)
         float vm = 0.f;
@@ -493,6 +513,7 @@ kv_decode_tc_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
             // ---- keys: convert, hand to the MMA warp
             dec_convert_row(krow, ktile, tid);
             load_row(kq, j + 1, krow);
+            prefetch_tile(j + 2);
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(bar_k);

@@ -102,9 +102,20 @@ kv_scores_tc_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
                 w[c] = make_uint4(0u, 0u, 0u, 0u);
         }
     };
+    // token t of local tile j, two tiles ahead of its register load: its code
+    // row and scale into L2
+    auto prefetch_tile = [&](int j) {
+        const int64_t t = (j0 + j) * kDecTile + tid;
+        if (j < ntiles && t < T) {
+            const int64_t r = (b * T + t) * Hkv + h;
+            prefetch_l2(kq + r * 64);
+            prefetch_l2(ks + r);
+        }
+    };
     uint4 krow[4];
     if (compute) {
         load_row(0, krow);
+        prefetch_tile(1);
         dec_rotate_queries<G>(q + (b * Hq + (int64_t)h * G) * 128, signs + h * 128, bq, inv_qs, tid);
     }
     fence_proxy_async_smem();
@@ -175,6 +186,7 @@ kv_scores_tc_kernel(const __half *__restrict__ q,        // [B, Hq, 128]
             // buffer, were waited for in the previous iteration), hand over
             dec_convert_row(krow, tile_of(j), tid);
             load_row(j + 1, krow);
+            prefetch_tile(j + 2);
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(bar_k(j));
